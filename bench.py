@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of the deterministic-reduction hot path on B200.
+
+One step = one pass over every kernel of the path on seeded synthetic inputs
+shaped like the pages' workloads:
+  plan      stable sort of 4096 tokens by adapter id (8 adapters)
+  shrink    segmented LoRA shrink, M=4096, K=4096, r=16, split-K 8:
+            tree (deterministic), atomic, unsplit
+  expand    segmented LoRA expand r=16 -> N=4096
+  shrink16  LoRA shrink M=16, K=4096, r=16: tree s=8, atomic s=8, unsplit
+  gemm      batch-invariant GEMM M=4096, N=4096, K=4096 (tcgen05)
+  treegemm  TP-invariant tree GEMM M=2048, N=4096, K=16384, 8 emulated shards
+  rmsnorm   4096 x 4096 bf16
+  lsm       log_softmax 4096 x 151936 fp32
+  mean      mean of the same 4096 x 151936 fp32 rows
+
+The headline `value` is the deterministic split-K LoRA-shrink HBM GB/s on
+the segmented workload (algorithmic bytes / kernel time, CUDA events on the
+launch stream).  Every kernel's own time, throughput and roofline fraction
+is listed under "kernels"; "roofline" describes the kernel with the largest
+share of the step.  L2 is flushed (a 256 MiB memset) before each kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Det. split-K LoRA-shrink HBM GB/s; BI-GEMM TFLOP/s; % of roofline; Δ vs atomic"
+WORKLOAD = ("segmented multi-adapter LoRA shrink M=4096 tokens, 8 adapters, K=4096, r=16, "
+            "split-K 8 tree, inside one pass of the whole deterministic-reduction path")
+L2_FLUSH_BYTES = 256 << 20
+
+# shrink algorithmic bytes (segmented, r=16): x + A + y + plan(perm + offsets)
+M4, K4, R4, NAD = 4096, 4096, 16, 8
+SHRINK_BYTES = M4 * K4 * 2 + NAD * R4 * K4 * 2 + M4 * R4 * 4 + 4 * (M4 + NAD + 2)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+class Workload:
+    """Device-resident inputs and outputs of one step, and its kernel list."""
+
+    def __init__(self, bi, synth, seed):
+        self.bi = bi
+        d = synth.lora_inputs(M4, K4, R4, n_adapters=NAD, N=4096, seed=seed)
+        self.ids_host = d["ids"]
+        self.x_host = d["x"]
+        self.x = dev_bf16(d["x"])
+        self.A = dev_bf16(d["at"])
+        self.B = dev_bf16(d["bt"])
+        self.ids = torch.from_numpy(d["ids"]).cuda()
+        self.plan = torch.empty(bi.lora_plan_bytes(M4, NAD) // 4, dtype=torch.int32, device="cuda")
+        self.y = torch.empty(M4, R4, dtype=torch.float32, device="cuda")
+        self.y_at = torch.empty_like(self.y)
+        self.y_un = torch.empty_like(self.y)
+        self.out = torch.empty(M4, 4096, dtype=torch.float32, device="cuda")
+        d1 = synth.lora_inputs(16, 4096, 16, seed=seed)
+        self.x16, self.A16 = dev_bf16(d1["x"]), dev_bf16(d1["at"][0])
+        self.y16 = torch.empty(16, 16, dtype=torch.float32, device="cuda")
+        xr, wr = synth.rmsnorm_inputs(4096, 4096, seed=seed)
+        self.xr, self.wr = dev_bf16(xr), dev_bf16(wr)
+        self.yr = torch.empty_like(self.xr)
+        self.logits = torch.from_numpy(synth.logits_inputs(4096, 151936, seed=seed)).cuda()
+        self.lsm = torch.empty_like(self.logits)
+        self.mean = torch.empty(4096, dtype=torch.float32, device="cuda")
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.kernels = self._kernels()
+
+    def _kernels(self):
+        """(name, fn, algorithmic bytes, flops, bound, our launches per call)"""
+        bi = self.bi
+        lsm_bytes = 4096 * 151936 * 8
+        k = [
+            ("plan", lambda: bi.lora_plan(self.ids, NAD, self.plan), 4 * M4 + 4 * (M4 + NAD + 2), 0, "hbm", 1),
+            ("shrink_tree_s8", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y, 8, "tree"),
+             SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
+            ("shrink_atomic_s8", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y_at, 8, "atomic"),
+             SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
+            ("shrink_unsplit", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y_un, 1, "unsplit"),
+             SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
+            ("expand", lambda: bi.lora_expand_segmented(self.y, self.B, self.plan, self.out),
+             M4 * R4 * 4 + NAD * 4096 * R4 * 2 + M4 * 4096 * 4 + 4 * M4, 2 * M4 * 4096 * R4, "hbm", 1),
+            ("shrink16_tree_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "tree"),
+             16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
+            ("shrink16_atomic_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "atomic"),
+             16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
+            ("shrink16_unsplit", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 1, "unsplit"),
+             16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
+            ("rmsnorm", lambda: bi.rmsnorm(self.xr, self.wr, self.yr, 1e-6),
+             4096 * 4096 * 4 + 4096 * 2, 0, "hbm", 1),
+            ("log_softmax", lambda: bi.log_softmax(self.logits, self.lsm), lsm_bytes, 0, "hbm", 1),
+            ("mean", lambda: bi.mean(self.logits, self.mean), 4096 * 151936 * 4 + 4096 * 4, 0, "hbm", 1),
+        ]
+        k += self._gemm_kernels()
+        return k
+
+    def _gemm_kernels(self):
+        bi = self.bi
+        out = []
+        try:
+            M, N, K = 4096, 4096, 4096
+            import invariant_bi_lora_b200.synth as synth
+            a, w = synth.gemm_inputs(M, N, K, seed=0)
+            self.ga, self.gw = dev_bf16(a), dev_bf16(w)
+            self.gc = torch.empty(M, N, dtype=torch.float32, device="cuda")
+            bi.gemm(self.ga, self.gw, self.gc)
+            out.append(("gemm", lambda: bi.gemm(self.ga, self.gw, self.gc), 2 * M * K + 2 * N * K + 4 * M * N,
+                        2 * M * N * K, "tensor", 1))
+        except bi.BiError:
+            pass
+        try:
+            M, N, K, S = 2048, 4096, 16384, 8
+            import invariant_bi_lora_b200.synth as synth
+            a, w = synth.gemm_inputs(M, N, K, seed=1)
+            self.ta, self.tw = dev_bf16(a), dev_bf16(w)
+            self.tc = torch.empty(M, N, dtype=torch.float32, device="cuda")
+            self.tws = torch.empty(bi.gemm_tree_ws_bytes(M, N, S), dtype=torch.uint8, device="cuda")
+            bi.gemm_tree(self.ta, self.tw, self.tc, S, self.tws)
+            out.append(("tree_gemm_s8", lambda: bi.gemm_tree(self.ta, self.tw, self.tc, S, self.tws),
+                        2 * M * K + 2 * N * K + 4 * M * N, 2 * M * N * K, "tensor", 2))
+        except bi.BiError:
+            pass
+        return out
+
+
+def run_ours(args, rank, world, device):
+    from invariant_bi_lora_b200 import bi, synth
+    wl = Workload(bi, synth, seed=0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    def step(events=None):
+        for i, (name, fn, *_rest) in enumerate(wl.kernels):
+            wl.flush.fill_(i & 0xff)               # L2 flush: 256 MiB write
+            if events is not None:
+                events[i][0].record(stream)
+            fn()
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if bi.get_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    nk = len(wl.kernels)
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for s in range(args.steps):
+        step(ev[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    per = {name: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
+           for i, (name, *_r) in enumerate(wl.kernels)}
+    if world > 1:
+        t = torch.tensor([total_ms] + [sum(v) for v in per.values()], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t[0])
+        for j, k in enumerate(per):
+            scale = float(t[j + 1]) / max(sum(per[k]), 1e-9)
+            per[k] = [v * scale for v in per[k]]
+    status = bi.get_device_status()
+
+    kern = []
+    for (name, fn, nbytes, flops, bound, launches) in wl.kernels:
+        ms = statistics.mean(per[name])
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tfl = flops / (ms * 1e-3) / 1e12 if flops else None
+        if bound == "tensor":
+            ach, peak, unit = tfl, pk["bf16_tflops_sustained"], "TFLOP/s"
+        else:
+            ach, peak, unit = gbs, pk["hbm_gbs"], "GB/s"
+        kern.append({"name": name, "us": round(ms * 1e3, 3), "bytes": nbytes, "flops": flops,
+                     "gbs": round(gbs, 1), "tflops": None if tfl is None else round(tfl, 2),
+                     "bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
+                     "frac": round(ach / peak, 4), "launches": launches})
+    by = {k["name"]: k for k in kern}
+    dom = max(kern, key=lambda k: k["us"])
+    tree = by["shrink_tree_s8"]
+    value = world * tree["gbs"]
+    gemm = by.get("gemm")
+    e2e = measure_e2e(wl, bi, args) if rank == 0 else None
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy PCG64; shapes of the pages' workloads)",
+        "config": {"workload": WORKLOAD, "global_batch": M4 * world, "seq_len": None,
+                   "parallelism": f"dp{world} (independent replicas, no collective)",
+                   "l2": "flushed before every kernel (256 MiB write)"},
+        "roofline": {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"],
+                     "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
+                     "traffic": None, "peak_source": pk["source"]},
+        "shrink_roofline": {"bound": "hbm", "achieved": tree["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": tree["frac"], "bytes_per_launch": SHRINK_BYTES},
+        "delta_vs_atomic_pct": round(100.0 * (tree["us"] / by["shrink_atomic_s8"]["us"] - 1.0), 2),
+        "speedup_vs_unsplit_pct": round(100.0 * (by["shrink_unsplit"]["us"] / tree["us"] - 1.0), 2),
+        "bi_gemm_tflops": None if gemm is None else gemm["tflops"],
+        "kernels": kern,
+        "gpu_launches": args.steps * sum(k["launches"] for k in kern),
+        "device_status": status,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return line
+
+
+def measure_e2e(wl, bi, args):
+    """Same metric through the public API with host buffers: every step
+    copies x and the adapter ids from pinned host memory, builds the plan,
+    runs the deterministic shrink and reads y back to the host."""
+    x_h = torch.from_numpy(np.ascontiguousarray(wl.x_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+    ids_h = torch.from_numpy(wl.ids_host).pin_memory()
+    y_h = torch.empty(M4, R4, dtype=torch.float32).pin_memory()
+    x_d = torch.empty_like(wl.x)
+    ids_d = torch.empty_like(wl.ids)
+    stream = torch.cuda.current_stream()
+
+    def one():
+        x_d.copy_(x_h, non_blocking=True)
+        ids_d.copy_(ids_h, non_blocking=True)
+        bi.lora_plan(ids_d, NAD, wl.plan)
+        bi.lora_shrink_segmented(x_d, wl.A, wl.plan, wl.y, 8, "tree")
+        y_h.copy_(wl.y, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(args.steps, 10)
+    a.record(stream)
+    for _ in range(n):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    return {"value": round(SHRINK_BYTES / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": x_h.numel() * 2 + ids_h.numel() * 4,
+            "d2h_bytes_per_step": y_h.numel() * 4, "ms_per_step": round(ms, 4)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_shrink_rate(seconds=10.0):
+    """The oracle's fp64 shrink over the segmented workload (all 4096
+    tokens, 8 adapters), repeated for about `seconds`; returns GB/s in the
+    same algorithmic-bytes unit, threads used, passes."""
+    import oracle
+    from invariant_bi_lora_b200 import synth
+    d = synth.lora_inputs(M4, K4, R4, n_adapters=NAD, seed=0)
+    nt = oracle.max_threads()
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        oracle.shrink_exact(d["x"], d["at"], d["ids"], nthreads=nt)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return SHRINK_BYTES * passes / el / 1e9, nt, passes, el
+
+
+def cpu_baseline_entry(seconds):
+    v, nt, passes, el = oracle_shrink_rate(seconds)
+    return {"value": round(v, 3), "unit": "GB/s", "cores": nt, "kind": "oracle",
+            "sample": f"{passes} full passes of the oracle's fp64 shrink over the segmented "
+                      f"workload (4096 tokens x 4096 x r=16, 8 adapters) in {el:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    from invariant_bi_lora_b200 import synth
+    d = synth.lora_inputs(M4, K4, R4, n_adapters=NAD, seed=0)
+    nt = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle.shrink_exact(d["x"][:256], d["at"], d["ids"][:256], nthreads=nt)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.shrink_exact(d["x"], d["at"], d["ids"], nthreads=nt)
+    el = time.perf_counter() - t0
+    v = SHRINK_BYTES * args.steps / el / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": M4, "seq_len": None, "parallelism": "cpu"},
+            "cpu_baseline": {"value": round(v, 3), "unit": "GB/s", "cores": nt, "kind": "oracle",
+                             "sample": f"{args.steps} full passes of the oracle's fp64 segmented shrink"},
+            "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    # CPU baseline first (rank 0, N=1 only), before any GPU work.
+    cpu = cpu_baseline_entry(args.cpu_seconds) if (rank == 0 and world == 1) else None
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,106 @@
+// combine.cu -- cross-shard combine of tensor-parallel partials.
+//
+// "Deterministic Inference across Tensor Parallel Sizes That Eliminates
+// Training-Inference Mismatch" (Abstract): the inter-GPU reduction follows
+// the same hierarchical binary tree as the intra-GPU one.  With K split into
+// s contiguous shards that are subtrees of the canonical tree, the shard
+// partials are combined by the top levels of that tree: out[i] =
+// tree(partials[0][i], ..., partials[s-1][i]).  The tree is evaluated in
+// post order on a small register stack (the merge schedule is computed on
+// the host), four elements per thread with 16-byte loads.
+#include "common.cuh"
+
+#include <algorithm>
+
+namespace bi {
+
+constexpr int kMaxCombine = 64;
+
+struct CombineParams {
+  const float *parts;
+  float *out;
+  size_t count;
+  int s;
+  uint8_t merges[kMaxCombine];
+};
+
+__global__ void __launch_bounds__(256)
+tree_combine_kernel(const __grid_constant__ CombineParams p) {
+  constexpr int D = 7;   // stack depth for s <= 64
+  const size_t nv = p.count / 4;
+  const float4 *src = reinterpret_cast<const float4 *>(p.parts);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 st[D];
+#pragma unroll
+    for (int d = 0; d < D; d++) st[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+    int depth = 0;
+    for (int j = 0; j < p.s; j++) {
+      const float4 v = __ldcs(src + (size_t)j * nv + i);
+#pragma unroll
+      for (int d = 0; d < D; d++) {
+        const bool hit = d == depth;
+        st[d].x = hit ? v.x : st[d].x;
+        st[d].y = hit ? v.y : st[d].y;
+        st[d].z = hit ? v.z : st[d].z;
+        st[d].w = hit ? v.w : st[d].w;
+      }
+      depth++;
+      const int nm = p.merges[j];
+#pragma unroll 1
+      for (int m = 0; m < nm; m++) {
+#pragma unroll
+        for (int d = 1; d < D; d++) {
+          const bool hit = d == depth - 1;
+          const float4 a = st[d - 1], b = st[d];
+          st[d - 1].x = hit ? __fadd_rn(a.x, b.x) : a.x;
+          st[d - 1].y = hit ? __fadd_rn(a.y, b.y) : a.y;
+          st[d - 1].z = hit ? __fadd_rn(a.z, b.z) : a.z;
+          st[d - 1].w = hit ? __fadd_rn(a.w, b.w) : a.w;
+        }
+        depth--;
+      }
+    }
+    reinterpret_cast<float4 *>(p.out)[i] = st[0];
+  }
+}
+
+// Post-order merge schedule of the canonical halving tree over n leaves.
+void tree_schedule(int n, uint8_t *merges) {
+  std::fill(merges, merges + n, 0);
+  struct R {
+    static void go(int lo, int hi, uint8_t *m) {
+      if (hi - lo <= 1) return;
+      const int h = lo + (hi - lo + 1) / 2;
+      go(lo, h, m);
+      go(h, hi, m);
+      m[hi - 1]++;
+    }
+  };
+  R::go(0, n, merges);
+}
+
+bi_status tree_combine_launch(const float *partials, float *out, int s, size_t count,
+                              cudaStream_t stream) {
+  if (s < 1 || s > kMaxCombine) return BI_ERR_INVALID_ARG;
+  if (count > 0 && (!partials || !out)) return BI_ERR_INVALID_ARG;
+  if (count % 4 != 0 || !bi_aligned16(partials) || !bi_aligned16(out)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (count == 0) return BI_OK;
+  CombineParams p{};
+  p.parts = partials;
+  p.out = out;
+  p.count = count;
+  p.s = s;
+  tree_schedule(s, p.merges);
+  const size_t nv = count / 4;
+  const unsigned blocks = (unsigned)std::min<size_t>((nv + 255) / 256, 148 * 8);
+  tree_combine_kernel<<<blocks, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace bi
+
+extern "C" bi_status bi_tree_combine(const float *partials, float *out, int s, size_t count,
+                                     bi_stream_t stream) {
+  return bi::tree_combine_launch(partials, out, s, count, reinterpret_cast<cudaStream_t>(stream));
+}

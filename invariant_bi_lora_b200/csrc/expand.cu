@@ -1,0 +1,158 @@
+// expand.cu -- LoRA expand out (+)= bf16(y) . B^T, single or multi-adapter.
+//
+// "Reproducible LoRA Inference Through Deterministic Split-K Reduction"
+// (Q&A): LoRA is two low-rank multiplications; the shrink reduces over the
+// hidden size, the expand reduces over the rank r only.  With K = r (8..128)
+// there is nothing to split: each output element is one tensor-core MMA
+// chain over r, computed the same way whatever M is, so the expand is
+// batch-invariant as it stands.  It is bound by the fp32 write of `out`
+// (M x N x 4 bytes), so the kernel is shaped for stores: a CTA owns a
+// 64-row x 128-column output tile, each warp a 16 x 64 strip, each thread
+// writes full 32-byte sectors.
+#include "common.cuh"
+
+namespace bi {
+
+constexpr int kExpBM = 64;     // rows per CTA (4 MMA row tiles)
+constexpr int kExpBN = 128;    // columns per CTA
+constexpr int kExpThreads = 256;
+
+struct ExpandParams {
+  const float *y;           // [M][r] fp32
+  const uint16_t *bt;       // [n_ad][N][r] bf16
+  const int32_t *perm;      // nullptr: identity
+  const int32_t *offsets;   // [n_ad + 2] or nullptr
+  float *out;               // [M][N] fp32
+  int M, r, N, n_ad, accumulate;
+};
+
+// KS = number of k16 steps (r rounded up to 16, / 16).
+template <int KS>
+__global__ void __launch_bounds__(kExpThreads)
+expand_kernel(const __grid_constant__ ExpandParams p) {
+  __shared__ TileInfo s_tile;
+  if (threadIdx.x == 0) s_tile = resolve_tile(p.offsets, p.n_ad, p.M, blockIdx.y, kExpBM);
+  __syncthreads();
+  const TileInfo ti = s_tile;
+  if (ti.adapter < 0) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int mt = warp & 3;                       // row tile 0..3
+  const int nbase = blockIdx.x * kExpBN + (warp >> 2) * 64;
+  const int lr0 = mt * 16 + g, lr1 = lr0 + 8;
+  const bool v0 = lr0 < ti.rows, v1 = lr1 < ti.rows;
+  const int row0 = v0 ? tile_row(p.perm, ti, lr0) : 0;
+  const int row1 = v1 ? tile_row(p.perm, ti, lr1) : 0;
+
+  if (ti.adapter == p.n_ad) {                    // tokens without an adapter
+    if (!p.accumulate) {
+      for (int nt = 0; nt < 8; nt++) {
+        const int n = nbase + nt * 8 + 2 * c;
+        if (n >= p.N) break;
+        if (v0) *reinterpret_cast<float2 *>(p.out + (size_t)row0 * p.N + n) = make_float2(0.f, 0.f);
+        if (v1) *reinterpret_cast<float2 *>(p.out + (size_t)row1 * p.N + n) = make_float2(0.f, 0.f);
+      }
+    }
+    return;
+  }
+
+  // A fragments: bf16(y) rows g, g+8, k slots 2c, 2c+1, 2c+8, 2c+9 of each
+  // k16 step (zero past r).
+  uint32_t afr[KS][4];
+#pragma unroll
+  for (int s = 0; s < KS; s++) {
+    const int k0 = 16 * s + 2 * c, k1 = k0 + 8;
+    float2 a00 = make_float2(0.f, 0.f), a10 = a00, a01 = a00, a11 = a00;
+    if (v0 && k0 < p.r) a00 = *reinterpret_cast<const float2 *>(p.y + (size_t)row0 * p.r + k0);
+    if (v1 && k0 < p.r) a10 = *reinterpret_cast<const float2 *>(p.y + (size_t)row1 * p.r + k0);
+    if (v0 && k1 < p.r) a01 = *reinterpret_cast<const float2 *>(p.y + (size_t)row0 * p.r + k1);
+    if (v1 && k1 < p.r) a11 = *reinterpret_cast<const float2 *>(p.y + (size_t)row1 * p.r + k1);
+    afr[s][0] = pack_bf16x2(a00.x, a00.y);
+    afr[s][1] = pack_bf16x2(a10.x, a10.y);
+    afr[s][2] = pack_bf16x2(a01.x, a01.y);
+    afr[s][3] = pack_bf16x2(a11.x, a11.y);
+  }
+
+  const uint16_t *bad = p.bt + (size_t)ti.adapter * p.N * p.r;
+#pragma unroll 2
+  for (int nt = 0; nt < 8; nt++) {
+    const int n0 = nbase + nt * 8;
+    if (n0 >= p.N) break;
+    const uint16_t *brow = bad + (size_t)(n0 + g) * p.r;   // B[n0+g][.]
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < KS; s++) {
+      const int k0 = 16 * s + 2 * c, k1 = k0 + 8;
+      uint32_t b[2];
+      b[0] = k0 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k0)) : 0u;
+      b[1] = k1 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k1)) : 0u;
+      mma_bf16_16816(acc, afr[s], b, acc);
+    }
+    const int n = n0 + 2 * c;
+    if (v0) {
+      float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row0 * p.N + n);
+      float2 v = make_float2(acc[0], acc[1]);
+      if (p.accumulate) {
+        const float2 q = *o;
+        v.x = __fadd_rn(q.x, v.x);
+        v.y = __fadd_rn(q.y, v.y);
+      }
+      *o = v;
+    }
+    if (v1) {
+      float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row1 * p.N + n);
+      float2 v = make_float2(acc[2], acc[3]);
+      if (p.accumulate) {
+        const float2 q = *o;
+        v.x = __fadd_rn(q.x, v.x);
+        v.y = __fadd_rn(q.y, v.y);
+      }
+      *o = v;
+    }
+  }
+}
+
+bi_status expand_launch(const float *y, const void *B, const int32_t *perm, const int32_t *offsets,
+                        int n_ad, float *out, int M, int r, int N, int accumulate,
+                        cudaStream_t stream) {
+  if (M < 0 || r <= 0 || N <= 0 || n_ad < 1) return BI_ERR_INVALID_ARG;
+  if (M > 0 && (!y || !B || !out)) return BI_ERR_INVALID_ARG;
+  if (r % 8 != 0 || r > 128 || N % 8 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(y) || !bi_aligned16(B) || !bi_aligned16(out)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return BI_OK;
+  ExpandParams p{y, static_cast<const uint16_t *>(B), perm, offsets, out, M, r, N, n_ad,
+                 accumulate ? 1 : 0};
+  const int tiles = offsets ? (M + kExpBM - 1) / kExpBM + n_ad + 1 : (M + kExpBM - 1) / kExpBM;
+  dim3 grid((N + kExpBN - 1) / kExpBN, tiles);
+  const int ks = (r + 15) / 16;
+  switch (ks) {
+    case 1: expand_kernel<1><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 2: expand_kernel<2><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 3: expand_kernel<3><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 4: expand_kernel<4><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 5: expand_kernel<5><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 6: expand_kernel<6><<<grid, kExpThreads, 0, stream>>>(p); break;
+    case 7: expand_kernel<7><<<grid, kExpThreads, 0, stream>>>(p); break;
+    default: expand_kernel<8><<<grid, kExpThreads, 0, stream>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace bi
+
+extern "C" bi_status bi_lora_expand(const float *y, const void *B, float *out, int M, int r, int N,
+                                    int accumulate, bi_stream_t stream) {
+  return bi::expand_launch(y, B, nullptr, nullptr, 1, out, M, r, N, accumulate,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_lora_expand_segmented(const float *y, const void *B, const void *plan,
+                                              int n_adapters, float *out, int M, int r, int N,
+                                              int accumulate, bi_stream_t stream) {
+  if (M > 0 && !plan) return BI_ERR_INVALID_ARG;
+  if (n_adapters < 1 || n_adapters > 256) return BI_ERR_INVALID_ARG;
+  const int32_t *perm = static_cast<const int32_t *>(plan);
+  return bi::expand_launch(y, B, perm, perm + M, n_adapters, out, M, r, N, accumulate,
+                           reinterpret_cast<cudaStream_t>(stream));
+}

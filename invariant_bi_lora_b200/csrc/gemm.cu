@@ -1,0 +1,270 @@
+// gemm.cu -- batch-invariant bf16 GEMM on the 5th-generation tensor cores.
+//
+// "The biggest Mystery of LLMs have just been solved" (Batch-Variant vs.
+// Batch-Invariant): a batch-invariant matmul uses a locked kernel policy
+// instead of an auto-picker, so the reduction order never depends on the
+// batch.  "Restoring AI Reproducibility" (3-2): matmul stays data-parallel,
+// with one consistent reduction order.  "Batch Invariant Ops" (Highlighted
+// Details): torch.mm.
+//
+// Locked policy: every call, whatever M is, uses the same 128 x 256 output
+// tile, steps K from 0 to K in 64-wide stages, accumulates each output
+// element in one TMEM accumulator by tcgen05.mma (M=128, N=256, K=16, bf16
+// in, fp32 accumulate) and never splits K.  Row m of C is therefore the
+// same bits for every M; rows past M are zero-filled by TMA and dropped.
+//
+// Pipeline (persistent, one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A and W tiles into a 4-stage shared ring
+//               (128-byte swizzle; 48 KB a stage)
+//   warp 1      TMEM allocator and MMA issuer (one elected thread)
+//   warps 2..5  epilogue: TMEM -> registers -> global (fp32 or bf16),
+//               lane quadrant = warp % 4
+// Two 256-column TMEM accumulators let the epilogue of tile i overlap the
+// MMAs of tile i+1.  Every wait is bounded (tc.cuh).
+#include "tc.cuh"
+
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace bi {
+
+namespace gemm {
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;                   // 2 accumulators x 256
+constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+}  // namespace gemm
+
+struct GemmSmemTail {
+  uint64_t full[gemm::STAGES];
+  uint64_t empty[gemm::STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  uint32_t bail;
+};
+
+__global__ void __launch_bounds__(gemm::THREADS, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                 void *__restrict__ C, int M, int N, int K, int c_bf16, unsigned *status) {
+  using namespace gemm;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sa = smem;                                 // [STAGES][A_BYTES]
+  uint8_t *sb = smem + STAGES * A_BYTES;              // [STAGES][B_BYTES]
+  GemmSmemTail *tail = reinterpret_cast<GemmSmemTail *>(smem + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kblocks = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&tail->tfull[b], 1);
+      mbar_init(&tail->tempty[b], 4);
+    }
+    tail->bail = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+  volatile uint32_t *bail = &tail->bail;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
+        const int mb = tile % tiles_m, nb = tile / tiles_m;
+        for (int kb = 0; kb < kblocks; kb++) {
+          if (!mbar_wait(&tail->empty[stage], phase ^ 1)) {
+            flag_error(status, BI_ERR_TIMEOUT);
+            *bail = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
+          tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, kb * BK, mb * BM);
+          tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, kb * BK, nb * BN);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
+        if (!mbar_wait(&tail->tempty[acc], acc_phase ^ 1)) {
+          flag_error(status, BI_ERR_TIMEOUT);
+          *bail = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < kblocks; kb++) {
+          if (!mbar_wait(&tail->full[stage], phase)) {
+            flag_error(status, BI_ERR_TIMEOUT);
+            *bail = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sa + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sb + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; k++)
+            umma_bf16(d, umma_desc_kmajor_sw128(a0 + 32 * k), umma_desc_kmajor_sw128(b0 + 32 * k), idesc,
+                      (kb | k) != 0);
+          umma_commit(&tail->empty[stage]);          // stage reusable once these MMAs finish
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        umma_commit(&tail->tfull[acc]);              // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // ---------------- epilogue: 4 warps, one TMEM lane quadrant each
+    const int quad = warp & 3;
+    const int row_in_tile = 32 * quad + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (*bail) break;
+      if (!mbar_wait(&tail->tfull[acc], acc_phase)) {
+        flag_error(status, BI_ERR_TIMEOUT);
+        *bail = 1;
+        break;
+      }
+      tc_fence_after();
+      const int mb = tile % tiles_m, nb = tile / tiles_m;
+      const int row = mb * BM + row_in_tile;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ch++) {
+        uint32_t v[32];
+        tmem_ld32(tbase + 32 * ch, v);
+        tmem_wait_ld();
+        const int col0 = nb * BN + 32 * ch;
+        if (row < M) {
+          if (!c_bf16) {
+            float *dst = static_cast<float *>(C) + (size_t)row * N + col0;
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+              if (col0 + 4 * j < N)
+                *reinterpret_cast<uint4 *>(dst + 4 * j) = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          } else {
+            uint16_t *dst = static_cast<uint16_t *>(C) + (size_t)row * N + col0;
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+              if (col0 + 8 * j < N) {
+                uint4 o;
+                o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                *reinterpret_cast<uint4 *>(dst + 8 * j) = o;
+              }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host
+
+static std::mutex g_tma_mu;
+
+bool make_tma_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_tma_mu);
+    if (!encode) {
+      void *fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bi_status gemm_launch(const void *A, const void *W, void *C, int M, int N, int K, int c_bf16,
+                      cudaStream_t stream) {
+  using namespace gemm;
+  if (M < 0 || N <= 0 || K <= 0) return BI_ERR_INVALID_ARG;
+  if (M > 0 && (!A || !W || !C)) return BI_ERR_INVALID_ARG;
+  if (K % BK != 0 || N % 16 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(A) || !bi_aligned16(W) || !bi_aligned16(C)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return BI_OK;
+  CUtensorMap tmA, tmW;
+  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
+  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) != cudaSuccess)
+      return BI_ERR_CUDA;
+    attr_set = true;
+  }
+  const long tiles = (long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)std::min<long>(tiles, num_sms());
+  gemm_bf16_kernel<<<grid, THREADS, SMEM, stream>>>(tmA, tmW, C, M, N, K, c_bf16 ? 1 : 0, status_word());
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace bi
+
+extern "C" bi_status bi_gemm(const void *A, const void *W, void *C, int M, int N, int K, int c_bf16,
+                             bi_stream_t stream) {
+  return bi::gemm_launch(A, W, C, M, N, K, c_bf16, reinterpret_cast<cudaStream_t>(stream));
+}

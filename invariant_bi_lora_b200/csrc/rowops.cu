@@ -1,0 +1,328 @@
+// rowops.cu -- batch-invariant RMSNorm, log_softmax and mean.
+//
+// "Restoring AI Reproducibility" (2-3, 3-1): RMSNorm contains a reduction,
+// and stays batch-invariant when each batch element is reduced by its own
+// core in a consistent order.  "Batch Invariant Ops" (Highlighted Details):
+// log_softmax and mean are among the ops made batch-invariant.
+//
+// One CTA (or one thread-block cluster) per row; the work of a row never
+// depends on how many rows the launch has.  The row sum is the canonical
+// lane sum: T logical lanes, lane t chains (from +0, in order) the V
+// elements of vectors t, t+T, t+2T, ..., and the T lane values are combined
+// by the canonical tree -- inside a warp by the xor butterfly 1,2,4,8,16
+// (which is that tree), across warps and CTAs by perfect trees over
+// power-of-two counts.  Vectors are 16 bytes: V = 8 for bf16, V = 4 for fp32.
+#include "bimath.cuh"
+
+#include <cooperative_groups.h>
+#include <algorithm>
+
+namespace cg = cooperative_groups;
+
+namespace bi {
+
+// ======================================================================
+// RMSNorm: T = 512 lanes of V = 8 bf16; one CTA of 512 threads per row,
+// thread t = lane t.  The row stays in registers (VPL vectors per lane)
+// between the sum and the scaling, so x is read from HBM once.
+// ======================================================================
+constexpr int kNormT = 512;
+
+template <int VPL>
+__global__ void __launch_bounds__(kNormT)
+rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
+               uint16_t *__restrict__ y, int n, float eps) {
+  __shared__ float s_warp[kNormT / 32];
+  __shared__ float s_inv;
+  const int t = threadIdx.x;
+  const size_t row = blockIdx.x;
+  const int nvec = n / 8;
+  const uint16_t *xr = x + row * n;
+
+  uint4 v[VPL];
+  float p = 0.0f;
+#pragma unroll
+  for (int j = 0; j < VPL; j++) {
+    const int vi = t + j * kNormT;
+    if (vi < nvec) {
+      v[j] = ldg128_stream(xr + 8 * vi);
+      const uint32_t q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const float a = bf16lo(q[e]), b = bf16hi(q[e]);
+        p = __fadd_rn(p, __fmul_rn(a, a));
+        p = __fadd_rn(p, __fmul_rn(b, b));
+      }
+    }
+  }
+  p = warp_tree_sum(p);
+  if ((t & 31) == 0) s_warp[t >> 5] = p;
+  __syncthreads();
+  if (t < 32) {
+    float q = t < kNormT / 32 ? s_warp[t] : 0.0f;
+#pragma unroll
+    for (int o = 1; o < kNormT / 32; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+    if (t == 0) {
+      const float ms = __fdiv_rn(q, (float)n);
+      s_inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    }
+  }
+  __syncthreads();
+  const float inv = s_inv;
+  uint16_t *yr = y + row * n;
+#pragma unroll
+  for (int j = 0; j < VPL; j++) {
+    const int vi = t + j * kNormT;
+    if (vi < nvec) {
+      const uint4 wv = ldg128(w + 8 * vi);
+      const uint32_t q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const float lo = __fmul_rn(__fmul_rn(bf16lo(q[e]), inv), bf16lo(wq[e]));
+        const float hi = __fmul_rn(__fmul_rn(bf16hi(q[e]), inv), bf16hi(wq[e]));
+        o[e] = pack_bf16x2(lo, hi);
+      }
+      *reinterpret_cast<uint4 *>(yr + 8 * vi) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// ======================================================================
+// mean: T = 1024 lanes of V = 4 fp32.  One CTA of 256 threads per row;
+// thread u owns the four adjacent lanes 4u..4u+3 (a subtree of the lane
+// tree), so each step it reads 64 contiguous bytes.
+// ======================================================================
+constexpr int kLaneT = 1024;
+constexpr int kMeanThreads = 256;
+
+__global__ void __launch_bounds__(kMeanThreads)
+mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
+  __shared__ float s_warp[kMeanThreads / 32];
+  const int u = threadIdx.x;
+  const size_t row = blockIdx.x;
+  const int nvec = n / 4;
+  const float4 *xr = reinterpret_cast<const float4 *>(x + row * n);
+  float p[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int base = 0; base < nvec; base += kLaneT) {
+    float4 v[4];
+#pragma unroll
+    for (int l = 0; l < 4; l++) {
+      const int vi = base + 4 * u + l;
+      v[l] = vi < nvec ? __ldcs(xr + vi) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int l = 0; l < 4; l++) {
+      if (base + 4 * u + l < nvec) {
+        p[l] = __fadd_rn(p[l], v[l].x);
+        p[l] = __fadd_rn(p[l], v[l].y);
+        p[l] = __fadd_rn(p[l], v[l].z);
+        p[l] = __fadd_rn(p[l], v[l].w);
+      }
+    }
+  }
+  float s = __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
+  s = warp_tree_sum(s);
+  if ((u & 31) == 0) s_warp[u >> 5] = s;
+  __syncthreads();
+  if (u < 32) {
+    float q = u < kMeanThreads / 32 ? s_warp[u] : 0.0f;
+#pragma unroll
+    for (int o = 1; o < kMeanThreads / 32; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+    if (u == 0) out[row] = __fdiv_rn(q, (float)n);
+  }
+}
+
+// ======================================================================
+// log_softmax: T = 1024 lanes of V = 4 fp32, two passes over the row
+// (max; then the canonical sum of bi_exp(x - max)), then the write.  The
+// row is held on chip between the passes so HBM sees one read and one
+// write: a cluster of C CTAs shares the row, CTA q owning lanes
+// [q*1024/C, (q+1)*1024/C) -- a subtree of the lane tree -- and keeping
+// its lanes' vectors in shared memory (slot [j][tau] for vector
+// 1024*j + lane).  Maxima and sums meet through distributed shared memory.
+// ======================================================================
+struct LsmParams {
+  const float *x;
+  float *out;
+  int n;
+  int C;      // CTAs per row (cluster size), power of two
+  int J;      // vector slots per lane = ceil(n/4 / 1024)
+};
+
+__global__ void __launch_bounds__(1024)
+log_softmax_kernel(const __grid_constant__ LsmParams p) {
+  extern __shared__ float4 lsm_smem[];
+  __shared__ float s_red[32];
+  __shared__ float s_max, s_sum;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = p.C;
+  const int q = (int)cluster.block_rank();
+  const int lpc = kLaneT / C;                  // lanes (= threads) per CTA
+  const int tau = threadIdx.x;
+  const int lane_id = q * lpc + tau;           // logical lane
+  const size_t row = blockIdx.x / C;
+  const int nvec = p.n / 4;
+  const float4 *xr = reinterpret_cast<const float4 *>(p.x + row * p.n);
+  float4 *outr = reinterpret_cast<float4 *>(p.out + row * p.n);
+  const int nwarps = lpc / 32;
+
+  // ---- load this lane's vectors into its shared-memory slots; local max
+  float m = -INFINITY;
+  for (int j = 0; j < p.J; j++) {
+    const int vi = j * kLaneT + lane_id;
+    if (vi < nvec) {
+      const float4 v = __ldcs(xr + vi);
+      lsm_smem[j * lpc + tau] = v;
+      m = fmaxf(fmaxf(m, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+    }
+  }
+  m = warp_max(m);
+  if ((tau & 31) == 0) s_red[tau >> 5] = m;
+  __syncthreads();
+  if (tau < 32) {
+    float v = tau < nwarps ? s_red[tau] : -INFINITY;
+    v = warp_max(v);
+    if (tau == 0) s_max = v;
+  }
+  cluster.sync();
+  // row max over the cluster (max is exact in any order)
+  float rmax = -INFINITY;
+  for (int r = 0; r < C; r++) rmax = fmaxf(rmax, *cluster.map_shared_rank(&s_max, r));
+
+  // ---- lane chain of bi_exp(x - max)
+  float s = 0.0f;
+  for (int j = 0; j < p.J; j++) {
+    const int vi = j * kLaneT + lane_id;
+    if (vi < nvec) {
+      const float4 v = lsm_smem[j * lpc + tau];
+      s = __fadd_rn(s, bi_exp(__fsub_rn(v.x, rmax)));
+      s = __fadd_rn(s, bi_exp(__fsub_rn(v.y, rmax)));
+      s = __fadd_rn(s, bi_exp(__fsub_rn(v.z, rmax)));
+      s = __fadd_rn(s, bi_exp(__fsub_rn(v.w, rmax)));
+    }
+  }
+  s = warp_tree_sum(s);
+  __syncthreads();                      // s_red reuse
+  if ((tau & 31) == 0) s_red[tau >> 5] = s;
+  __syncthreads();
+  if (tau < 32) {
+    float v = tau < nwarps ? s_red[tau] : 0.0f;
+    for (int o = 1; o < nwarps; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (tau == 0) s_sum = v;
+  }
+  cluster.sync();
+  // perfect tree over the C CTA subtrees (every CTA computes the same bits)
+  float part[16];
+#pragma unroll
+  for (int r = 0; r < 16; r++) part[r] = r < C ? *cluster.map_shared_rank(&s_sum, r) : 0.0f;
+#pragma unroll
+  for (int st = 1; st < 16; st <<= 1)
+#pragma unroll
+    for (int r = 0; r + st < 16; r += 2 * st)
+      if (r + st < C) part[r] = __fadd_rn(part[r], part[r + st]);
+  const float L = bi_log(part[0]);
+
+  // ---- write out = (x - max) - L
+  for (int j = 0; j < p.J; j++) {
+    const int vi = j * kLaneT + lane_id;
+    if (vi < nvec) {
+      const float4 v = lsm_smem[j * lpc + tau];
+      float4 o;
+      o.x = __fsub_rn(__fsub_rn(v.x, rmax), L);
+      o.y = __fsub_rn(__fsub_rn(v.y, rmax), L);
+      o.z = __fsub_rn(__fsub_rn(v.z, rmax), L);
+      o.w = __fsub_rn(__fsub_rn(v.w, rmax), L);
+      __stcs(outr + vi, o);
+    }
+  }
+  cluster.sync();   // peers may still read s_max / s_sum of this CTA
+}
+
+// Test and reference hook: the library's exp / log applied elementwise.
+__global__ void math_spec_kernel(const float *__restrict__ x, float *__restrict__ y, size_t n,
+                                 int which) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    y[i] = which == 0 ? bi_exp(x[i]) : bi_log(x[i]);
+}
+
+}  // namespace bi
+
+// ----------------------------------------------------------------------
+extern "C" bi_status bi_rmsnorm(const void *x, const void *w, void *y, int rows, int n, float eps,
+                                bi_stream_t stream) {
+  if (rows < 0 || n <= 0) return BI_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !w || !y)) return BI_ERR_INVALID_ARG;
+  if (n % 8 != 0 || n > 8 * bi::kNormT * 8) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(x) || !bi_aligned16(w) || !bi_aligned16(y)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return BI_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int vpl = (n / 8 + bi::kNormT - 1) / bi::kNormT;
+  auto xp = static_cast<const uint16_t *>(x);
+  auto wp = static_cast<const uint16_t *>(w);
+  auto yp = static_cast<uint16_t *>(y);
+  if (vpl <= 1) bi::rmsnorm_kernel<1><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
+  else if (vpl <= 2) bi::rmsnorm_kernel<2><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
+  else if (vpl <= 4) bi::rmsnorm_kernel<4><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
+  else bi::rmsnorm_kernel<8><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+extern "C" bi_status bi_mean(const float *x, float *out, int rows, int n, bi_stream_t stream) {
+  if (rows < 0 || n <= 0) return BI_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !out)) return BI_ERR_INVALID_ARG;
+  if (n % 4 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(x)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return BI_OK;
+  bi::mean_kernel<<<rows, bi::kMeanThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, out, n);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n, bi_stream_t stream) {
+  if (rows < 0 || n <= 0) return BI_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !out)) return BI_ERR_INVALID_ARG;
+  if (n % 4 != 0 || n > 262144) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(x) || !bi_aligned16(out)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return BI_OK;
+  bi::LsmParams p{x, out, n, 1, 0};
+  const int nvec = n / 4;
+  p.J = (nvec + bi::kLaneT - 1) / bi::kLaneT;
+  // Smallest cluster whose per-CTA share of the row fits in ~80 KB of
+  // shared memory (two CTAs per SM), at most 16.  Bit-neutral.
+  int C = 1;
+  while (C < 16 && (size_t)p.J * (bi::kLaneT / C) * 16 > 80 * 1024) C *= 2;
+  p.C = C;
+  const size_t smem = (size_t)p.J * (bi::kLaneT / C) * 16;
+  if (smem > 200 * 1024) return BI_ERR_UNSUPPORTED_SHAPE;
+  cudaError_t e = cudaFuncSetAttribute(bi::log_softmax_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return BI_ERR_CUDA;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(bi::log_softmax_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows * C, 1, 1);
+  cfg.blockDim = dim3(bi::kLaneT / C, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, bi::log_softmax_kernel, p);
+  return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+extern "C" bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream) {
+  if ((n > 0 && (!x || !y)) || (which != 0 && which != 1)) return BI_ERR_INVALID_ARG;
+  if (n == 0) return BI_OK;
+  const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16);
+  bi::math_spec_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, which);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}

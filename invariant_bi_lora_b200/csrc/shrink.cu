@@ -1,0 +1,401 @@
+// shrink.cu -- LoRA shrink y = x . A with a fixed-order split-K reduction.
+//
+// "Reproducible LoRA Inference Through Deterministic Split-K Reduction"
+// (Highlights, Q&A): the split-K shrink of vLLM adds its K-partials with fp32
+// atomics, so identical inputs give different bits; a deterministic split-K
+// keeps the parallelism and combines the partials in a fixed order.
+// "Deterministic Inference across Tensor Parallel Sizes ..." (Abstract): one
+// hierarchical binary tree orders every level of the reduction.
+//
+// Reduction order (the same for every M, split count, tile shape, replay):
+//   leaf   = 64 consecutive k; its value is one chain of four m16n8k16
+//            tensor-core MMAs started from zero (the order inside an MMA is
+//            the hardware's, identical for every row and every call);
+//   leaves = combined by the canonical halving tree in fp32 (__fadd_rn).
+// A CTA owns a contiguous power-of-two block of leaves (one subtree).  Its
+// warps split that block into G contiguous groups (subtrees again); a warp
+// folds its group's leaves in post order on a register stack, the G group
+// values meet in shared memory (perfect tree), and in mode TREE the
+// `splits` CTAs of a row tile -- one thread-block cluster -- meet through
+// distributed shared memory, perfect tree again.  Every level is a level
+// of the one canonical tree over the K/64 leaves, so the bits cannot depend
+// on how the work was cut.
+//
+// Data path: both operands are K-contiguous (x [M][K], A [r][K]), so a
+// thread fetches the eight consecutive k of its fragment row with one
+// 128-bit load, for x and for A alike.  Inside a 32-wide k chunk, thread
+// (g, c) feeds k = 8c..8c+7 to MMA k-slots {2c, 2c+1, 2c+8, 2c+9} of two
+// MMAs; the same permutation is applied to both operands, so the products
+// summed are exactly x[m][k] * A[j][k].  No shared-memory staging: the loads
+// go straight to registers, one leaf ahead of the MMAs.
+#include "common.cuh"
+
+#include <cooperative_groups.h>
+#include <algorithm>
+#include <vector>
+
+namespace cg = cooperative_groups;
+
+namespace bi {
+
+constexpr int kLeaf = 64;          // k per leaf
+constexpr int kMaxGroupLeaves = 1024;
+constexpr int kMaxSplits = 16;
+
+struct ShrinkParams {
+  const uint16_t *x;        // [M][K] bf16
+  const uint16_t *at;       // [n_ad][r][K] bf16
+  const int32_t *perm;      // token order grouped by adapter (nullptr: identity)
+  const int32_t *offsets;   // [n_ad + 2] segment starts in perm (nullptr: one segment)
+  float *y;                 // [M][r] fp32
+  unsigned *status;
+  int M, K, r, n_ad;
+  int splits;               // CTAs per row tile (cluster width in mode TREE)
+  int lc;                   // leaves per CTA = K / 64 / splits
+  int groups;               // G: leaf groups per CTA (power of two, divides lc)
+  int lg;                   // leaves per group = lc / G
+  int mtiles;               // MT: 16-row MMA tiles per CTA
+  int ngroups;              // NG: rank groups of NGW columns
+  int mode;
+  uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
+};
+
+// A leaf's operand fragments: x rows g and g+8 and the NT A columns, for the
+// two 32-wide k chunks of the leaf.
+template <int NT>
+struct LeafFrag {
+  uint4 xa[2][2];     // [chunk][row g / row g+8]
+  uint4 ab[2][NT];    // [chunk][n-tile]
+};
+
+template <int NT>
+BI_DEV void load_leaf(LeafFrag<NT> &f, const uint16_t *xr0, const uint16_t *xr1, bool v0,
+                      bool v1, const uint16_t *const *acol, int k) {
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    const int kk = k + 32 * h;
+    f.xa[h][0] = v0 ? ldg128_stream(xr0 + kk) : make_uint4(0, 0, 0, 0);
+    f.xa[h][1] = v1 ? ldg128_stream(xr1 + kk) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int t = 0; t < NT; t++) f.ab[h][t] = ldg128(acol[t] + kk);
+  }
+}
+
+// One leaf: four MMAs per n-tile (two k chunks x two k16 steps), from zero.
+template <int NT>
+BI_DEV void mma_leaf(float acc[NT][4], const LeafFrag<NT> &f) {
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int q = 0; q < 4; q++) acc[t][q] = 0.0f;
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    const uint4 r0 = f.xa[h][0], r1 = f.xa[h][1];
+    const uint32_t a_s0[4] = {r0.x, r1.x, r0.y, r1.y};
+    const uint32_t a_s1[4] = {r0.z, r1.z, r0.w, r1.w};
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const uint4 b = f.ab[h][t];
+      const uint32_t b_s0[2] = {b.x, b.y};
+      const uint32_t b_s1[2] = {b.z, b.w};
+      mma_bf16_16816(acc[t], a_s0, b_s0, acc[t]);
+      mma_bf16_16816(acc[t], a_s1, b_s1, acc[t]);
+    }
+  }
+}
+
+template <int NGW, int MAXD>
+__global__ void __launch_bounds__(256)
+shrink_kernel(const __grid_constant__ ShrinkParams p) {
+  constexpr int NT = NGW / 8;
+  extern __shared__ float4 smem_f4[];
+  float *part = reinterpret_cast<float *>(smem_f4);     // [G][BM][r]
+  __shared__ TileInfo s_tile;
+
+  const int bm = 16 * p.mtiles;
+  const int split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+
+  if (threadIdx.x == 0) s_tile = resolve_tile(p.offsets, p.n_ad, p.M, blockIdx.y, bm);
+  __syncthreads();
+  const TileInfo ti = s_tile;
+  if (ti.adapter < 0) return;                       // uniform across the cluster
+
+  if (ti.adapter == p.n_ad) {                       // tokens without an adapter
+    if (p.mode != BI_SHRINK_ATOMIC && split == 0) {
+      for (int e = threadIdx.x; e < ti.rows * p.r; e += blockDim.x) {
+        const int pos = ti.seg_begin + ti.row0 + e / p.r;
+        p.y[(size_t)p.perm[pos] * p.r + e % p.r] = 0.0f;
+      }
+    }
+    return;
+  }
+
+  // ---- warp role: (leaf group, m-tile, rank group)
+  const int per_lg = p.mtiles * p.ngroups;
+  const int lgi = warp / per_lg;
+  const int mt = (warp % per_lg) / p.ngroups;
+  const int ng = warp % p.ngroups;
+
+  // rows g and g+8 of this warp's m-tile
+  const int lr0 = mt * 16 + g, lr1 = lr0 + 8;       // local rows in the tile
+  const bool v0 = lr0 < ti.rows, v1 = lr1 < ti.rows;
+  int row0 = 0, row1 = 0;
+  if (v0) row0 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr0] : ti.row0 + lr0;
+  if (v1) row1 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr1] : ti.row0 + lr1;
+  const uint16_t *xr0 = p.x + (size_t)row0 * p.K + 8 * c;
+  const uint16_t *xr1 = p.x + (size_t)row1 * p.K + 8 * c;
+  const uint16_t *acol[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+    acol[t] = p.at + ((size_t)ti.adapter * p.r + ng * NGW + t * 8 + g) * p.K + 8 * c;
+
+  // ---- this warp's leaves: [leaf0, leaf0 + lg), folded in post order
+  const int leaf0 = split * p.lc + lgi * p.lg;
+  float st[MAXD][NT][4];
+#pragma unroll
+  for (int d = 0; d < MAXD; d++)
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int q = 0; q < 4; q++) st[d][t][q] = 0.0f;
+  int depth = 0;
+
+  LeafFrag<NT> cur, nxt;
+  load_leaf<NT>(cur, xr0, xr1, v0, v1, acol, leaf0 * kLeaf);
+  for (int i = 0; i < p.lg; i++) {
+    if (i + 1 < p.lg) load_leaf<NT>(nxt, xr0, xr1, v0, v1, acol, (leaf0 + i + 1) * kLeaf);
+    float acc[NT][4];
+    mma_leaf<NT>(acc, cur);
+    // push (register stack: every index is a compile-time constant, the
+    // slot is chosen by predication)
+#pragma unroll
+    for (int d = 0; d < MAXD; d++) {
+      const bool hit = d == depth;
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) st[d][t][q] = hit ? acc[t][q] : st[d][t][q];
+    }
+    depth++;
+    // merge the subtrees that end at this leaf: left = st[depth-2]
+    const int nm = p.merges[i];
+#pragma unroll 1
+    for (int m = 0; m < nm; m++) {
+#pragma unroll
+      for (int d = 1; d < MAXD; d++) {
+        const bool hit = d == depth - 1;
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            const float sum = __fadd_rn(st[d - 1][t][q], st[d][t][q]);
+            st[d - 1][t][q] = hit ? sum : st[d - 1][t][q];
+          }
+      }
+      depth--;
+    }
+    cur = nxt;
+  }
+  if (depth != 1) flag_error(p.status, BI_ERR_INVALID_ARG);   // schedule inconsistent
+
+  // ---- group values -> shared memory, element (local row, column)
+  const int E = bm * p.r;
+#pragma unroll
+  for (int t = 0; t < NT; t++) {
+    const int col = ng * NGW + t * 8 + 2 * c;
+    float *dst = part + (size_t)lgi * E;
+    dst[lr0 * p.r + col] = st[0][t][0];
+    dst[lr0 * p.r + col + 1] = st[0][t][1];
+    dst[lr1 * p.r + col] = st[0][t][2];
+    dst[lr1 * p.r + col + 1] = st[0][t][3];
+  }
+  __syncthreads();
+  // perfect tree over the G groups, in place into group 0
+  for (int s = 1; s < p.groups; s <<= 1) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      for (int q = 0; q + s < p.groups; q += 2 * s)
+        part[(size_t)q * E + e] = __fadd_rn(part[(size_t)q * E + e], part[(size_t)(q + s) * E + e]);
+    __syncthreads();
+  }
+
+  auto out_index = [&](int e) -> size_t {
+    const int lr = e / p.r;
+    const int row = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr] : ti.row0 + lr;
+    return (size_t)row * p.r + (e % p.r);
+  };
+  const int valid_E = ti.rows * p.r;
+
+  if (p.mode == BI_SHRINK_ATOMIC) {
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) atomicAdd(p.y + out_index(e), part[e]);
+    return;
+  }
+  if (p.splits == 1) {
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) p.y[out_index(e)] = part[e];
+    return;
+  }
+
+  // ---- mode TREE: the splits CTAs of this tile form one cluster; rank q
+  // holds the subtree of leaves [q*lc, (q+1)*lc).  Each CTA finishes a
+  // strided share of the elements: perfect tree over the ranks via DSMEM.
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  const int S = p.splits;
+  const float *peer[kMaxSplits];
+#pragma unroll
+  for (int q = 0; q < kMaxSplits; q++)
+    peer[q] = q < S ? cluster.map_shared_rank(part, q) : part;
+  for (int e = split * blockDim.x + threadIdx.x; e < valid_E; e += S * blockDim.x) {
+    float v[kMaxSplits];
+#pragma unroll
+    for (int q = 0; q < kMaxSplits; q++) v[q] = q < S ? peer[q][e] : 0.0f;
+#pragma unroll
+    for (int s = 1; s < kMaxSplits; s <<= 1)
+#pragma unroll
+      for (int q = 0; q + s < kMaxSplits; q += 2 * s)
+        if (q + s < S) v[q] = __fadd_rn(v[q], v[q + s]);
+    p.y[out_index(e)] = v[0];
+  }
+  cluster.sync();   // keep this CTA's shared memory alive until peers are done
+}
+
+// ----------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------
+
+// Post-order merge schedule of the canonical tree over n leaves: after leaf
+// i is pushed, merges[i] internal nodes end there.  Returns the largest
+// stack depth reached.
+static int tree_merge_schedule(int n, uint8_t *merges) {
+  std::fill(merges, merges + n, 0);
+  struct Rec {
+    static void go(int lo, int hi, uint8_t *m) {
+      if (hi - lo <= 1) return;
+      const int h = lo + (hi - lo + 1) / 2;
+      go(lo, h, m);
+      go(h, hi, m);
+      m[hi - 1]++;
+    }
+  };
+  Rec::go(0, n, merges);
+  int depth = 0, maxd = 0;
+  for (int i = 0; i < n; i++) {
+    depth++;
+    maxd = std::max(maxd, depth);
+    depth -= merges[i];
+  }
+  return maxd;
+}
+
+template <int NGW, int MAXD>
+static cudaError_t launch_shrink_t(const ShrinkParams &p, int tiles, int threads, size_t smem,
+                                   cudaStream_t stream) {
+  auto kern = shrink_kernel<NGW, MAXD>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, tiles, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  int na = 0;
+  if (p.mode == BI_SHRINK_TREE && p.splits > 1) {
+    if (p.splits > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    na = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// Validates, picks the (bit-neutral) tiling and launches.  perm/offsets are
+// null for the single-adapter call.
+bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const int32_t *offsets,
+                        int n_ad, float *y, int M, int K, int r, int splits, int mode,
+                        cudaStream_t stream) {
+  if (M < 0 || K <= 0 || r <= 0 || n_ad < 1) return BI_ERR_INVALID_ARG;
+  if (mode != BI_SHRINK_UNSPLIT && mode != BI_SHRINK_ATOMIC && mode != BI_SHRINK_TREE)
+    return BI_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !A || !y)) return BI_ERR_INVALID_ARG;
+  if (K % kLeaf != 0 || r % 8 != 0 || r > 128) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int L = K / kLeaf;
+  if (mode == BI_SHRINK_UNSPLIT && splits != 1) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_pow2(splits) || splits > kMaxSplits || L % splits != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(x) || !bi_aligned16(A)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return BI_OK;
+
+  ShrinkParams p{};
+  p.x = static_cast<const uint16_t *>(x);
+  p.at = static_cast<const uint16_t *>(A);
+  p.perm = perm;
+  p.offsets = offsets;
+  p.y = y;
+  p.status = status_word();
+  p.M = M; p.K = K; p.r = r; p.n_ad = n_ad;
+  p.splits = splits;
+  p.mode = mode;
+  p.lc = L / splits;
+
+  const int ngw = (r % 16 == 0) ? 16 : 8;
+  p.ngroups = r / ngw;
+  // m-tiles per CTA: up to 4 (64 rows), fewer when the batch is small
+  int mt = std::min(4, (M + 15) / 16);
+  while (mt > 1 && mt * p.ngroups > 8) mt >>= 1;
+  if (p.ngroups > 8) return BI_ERR_UNSUPPORTED_SHAPE;
+  p.mtiles = mt;
+  // leaf groups: fill up to 8 warps, power of two dividing lc
+  int G = 1;
+  while (G * 2 * mt * p.ngroups <= 8 && p.lc % (G * 2) == 0) G *= 2;
+  p.groups = G;
+  p.lg = p.lc / G;
+  if (p.lg > kMaxGroupLeaves) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int depth = tree_merge_schedule(p.lg, p.merges);
+  const int warps = G * mt * p.ngroups;
+  const int threads = 32 * warps;
+  const int bm = 16 * mt;
+  const size_t smem = (size_t)G * bm * r * sizeof(float);
+  const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
+
+  if (mode == BI_SHRINK_ATOMIC) {
+    BI_CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)M * r * sizeof(float), stream));
+  }
+  cudaError_t e;
+  if (ngw == 16) {
+    if (depth <= 4) e = launch_shrink_t<16, 4>(p, tiles, threads, smem, stream);
+    else if (depth <= 8) e = launch_shrink_t<16, 8>(p, tiles, threads, smem, stream);
+    else e = launch_shrink_t<16, 12>(p, tiles, threads, smem, stream);
+  } else {
+    if (depth <= 4) e = launch_shrink_t<8, 4>(p, tiles, threads, smem, stream);
+    else if (depth <= 8) e = launch_shrink_t<8, 8>(p, tiles, threads, smem, stream);
+    else e = launch_shrink_t<8, 12>(p, tiles, threads, smem, stream);
+  }
+  return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace bi
+
+extern "C" bi_status bi_lora_shrink(const void *x, const void *A, float *y, int M, int K, int r,
+                                    int splits, int mode, bi_stream_t stream) {
+  return bi::shrink_launch(x, A, nullptr, nullptr, 1, y, M, K, r, splits, mode,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_lora_shrink_segmented(const void *x, const void *A, const void *plan,
+                                              int n_adapters, float *y, int M, int K, int r,
+                                              int splits, int mode, bi_stream_t stream) {
+  if (M > 0 && !plan) return BI_ERR_INVALID_ARG;
+  if (n_adapters < 1 || n_adapters > 256) return BI_ERR_INVALID_ARG;
+  const int32_t *perm = static_cast<const int32_t *>(plan);
+  const int32_t *offsets = perm + M;
+  return bi::shrink_launch(x, A, perm, offsets, n_adapters, y, M, K, r, splits, mode,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
