@@ -64,7 +64,10 @@ def peaks():
 # --------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    """nvidia-smi sampling (every 100 ms) of SM clocks and throttle reasons.
+    Started before the warm-up; only samples taken inside the timed window
+    are summarised (the nearest ones if the window is shorter than one
+    sampling period)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -73,12 +76,13 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
+        self.window = (0.0, 0.0)
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -87,19 +91,27 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        t0, t1 = self.window
+        inside = [ln for (t, ln) in self.lines if t0 <= t <= t1]
+        if not inside and self.lines:
+            inside = [min(self.lines, key=lambda tl: abs(tl[0] - 0.5 * (t0 + t1)))[1]]
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -113,7 +125,8 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window_s": round(t1 - t0, 3)}
 
 
 # ------------------------------------------------------------------ workload
@@ -223,6 +236,8 @@ def run_ours(args, rank, world, device):
             if events is not None:
                 events[i][1].record(stream)
 
+    clocks = ClockSampler(device)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -233,18 +248,19 @@ def run_ours(args, rank, world, device):
     ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
           for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
+    h0 = time.time()
     t0.record(stream)
     for s in range(args.steps):
         step(ev[s])
     t1.record(stream)
     torch.cuda.synchronize()
+    h1 = time.time()
     if world > 1:
         torch.distributed.barrier()
+    clocks.mark(h0, h1)
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     per = {name: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
@@ -392,7 +408,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

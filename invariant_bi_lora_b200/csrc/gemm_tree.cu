@@ -1,0 +1,305 @@
+// gemm_tree.cu -- tensor-parallel-invariant GEMM: C = A . W^T with the K
+// reduction ordered by one hierarchical binary tree.
+//
+// "Deterministic Inference across Tensor Parallel Sizes That Eliminates
+// Training-Inference Mismatch" (Abstract): with intra- and inter-GPU
+// reductions aligned on one hierarchical binary tree, the result is the
+// same bits for every TP size.
+//
+// Order: K is cut into leaves of 256.  A leaf is one TMEM accumulation of
+// sixteen tcgen05.mma (M=128, N=64, K=16), restarted from zero for every
+// leaf.  Leaves are combined in fp32 by the canonical tree.  A shard (an
+// emulated TP rank) owns a contiguous block of L/shards leaves -- one
+// subtree -- and writes its partial; bi_tree_combine adds the top levels.
+//
+// Per CTA (persistent, 320 threads): warp 0 issues TMA loads into an
+// 8-stage ring, warp 1 issues the MMAs into one of two 64-column TMEM leaf
+// buffers, warps 2..9 fold finished leaves into the pending stack of the
+// post-order tree walk.  The stack lives in TMEM too: 6 slots of 64 columns
+// (2 x 64 + 6 x 64 = 512 columns), enough for 64 leaves per shard.  Each
+// epilogue thread owns one row (its TMEM lane) and 32 of the 64 columns.
+#include "tc.cuh"
+
+#include <algorithm>
+
+namespace bi {
+
+bi_status tree_combine_launch(const float *partials, float *out, int s, size_t count, cudaStream_t stream);
+
+namespace tg {
+constexpr int BM = 128, BN = 64, BK = 64, LEAF = 256, STAGES = 8;
+constexpr int KB_PER_LEAF = LEAF / BK;                // 4
+constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                  // 8 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 24 KB
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 32 * (2 + EPI_WARPS);         // 320
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int STACK_SLOTS = 6;
+constexpr int MAX_LEAVES = 64;                        // per shard
+constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+}  // namespace tg
+
+struct TreeGemmParams {
+  float *out;          // shards == 1: C [M][N]; else partials [shards][M][N]
+  unsigned *status;
+  int M, N, K, shards, leaves;   // leaves per shard
+  uint8_t merges[tg::MAX_LEAVES];
+};
+
+struct TreeSmemTail {
+  uint64_t full[tg::STAGES];
+  uint64_t empty[tg::STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  uint32_t bail;
+};
+
+__global__ void __launch_bounds__(tg::THREADS, 1)
+gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                 const __grid_constant__ TreeGemmParams p) {
+  using namespace tg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sa = smem;
+  uint8_t *sb = smem + STAGES * A_BYTES;
+  TreeSmemTail *tail = reinterpret_cast<TreeSmemTail *>(smem + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (p.M + BM - 1) / BM, tiles_n = p.N / BN;
+  const int num_tiles = tiles_m * tiles_n * p.shards;
+  const int L = p.leaves;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&tail->tfull[b], 1);
+      mbar_init(&tail->tempty[b], EPI_WARPS);
+    }
+    tail->bail = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+  volatile uint32_t *bail = &tail->bail;
+
+  // tile -> (m block, n block, shard); m fastest so concurrent CTAs share W
+  auto decode = [&](int t, int &mb, int &nb, int &sh) {
+    mb = t % tiles_m;
+    t /= tiles_m;
+    nb = t % tiles_n;
+    sh = t / tiles_n;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
+        int mb, nb, sh;
+        decode(tile, mb, nb, sh);
+        const int kb0 = sh * L * KB_PER_LEAF;
+        for (int kb = 0; kb < L * KB_PER_LEAF; kb++) {
+          if (!mbar_wait(&tail->empty[stage], phase ^ 1)) {
+            flag_error(p.status, BI_ERR_TIMEOUT);
+            *bail = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
+          tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, (kb0 + kb) * BK, mb * BM);
+          tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, (kb0 + kb) * BK, nb * BN);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t buf_phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
+        for (int leaf = 0; leaf < L && !*bail; leaf++) {
+          if (!mbar_wait(&tail->tempty[buf], buf_phase ^ 1)) {
+            flag_error(p.status, BI_ERR_TIMEOUT);
+            *bail = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(buf * BN);
+          for (int kb = 0; kb < KB_PER_LEAF; kb++) {
+            if (!mbar_wait(&tail->full[stage], phase)) {
+              flag_error(p.status, BI_ERR_TIMEOUT);
+              *bail = 1;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sa + stage * A_BYTES);
+            const uint32_t b0 = smem_u32(sb + stage * B_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; k++)
+              umma_bf16(d, umma_desc_kmajor_sw128(a0 + 32 * k), umma_desc_kmajor_sw128(b0 + 32 * k), idesc,
+                        (kb | k) != 0);                     // every leaf restarts from zero
+            umma_commit(&tail->empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          umma_commit(&tail->tfull[buf]);
+          if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: post-order fold of the leaves
+    const int ew = warp - 2;
+    const int quad = warp & 3;                  // TMEM lane quadrant of this warp
+    const int half = ew >> 2;                   // which 32 of the 64 columns
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    const uint32_t col_off = (uint32_t)(32 * half);
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (*bail) break;
+      int mb, nb, sh;
+      decode(tile, mb, nb, sh);
+      int top = 0;
+      for (int leaf = 0; leaf < L; leaf++) {
+        if (!mbar_wait(&tail->tfull[buf], buf_phase)) {
+          flag_error(p.status, BI_ERR_TIMEOUT);
+          *bail = 1;
+          break;
+        }
+        tc_fence_after();
+        uint32_t cur[32];
+        tmem_ld32(tmem + lane_off + (uint32_t)(buf * BN) + col_off, cur);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->tempty[buf]);
+        if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+        // subtrees that end at this leaf: cur = left + cur, left popped
+        for (int m = p.merges[leaf]; m > 0; m--) {
+          top--;
+          uint32_t left[32];
+          tmem_ld32(tmem + lane_off + (uint32_t)(2 * BN + top * BN) + col_off, left);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i++)
+            cur[i] = __float_as_uint(__fadd_rn(__uint_as_float(left[i]), __uint_as_float(cur[i])));
+        }
+        if (leaf + 1 < L) {
+          tmem_st32(tmem + lane_off + (uint32_t)(2 * BN + top * BN) + col_off, cur);
+          tmem_wait_st();
+          top++;
+        } else {
+          const int row = mb * BM + 32 * quad + lane;
+          if (row < p.M) {
+            float *dst = p.out + ((size_t)sh * p.M + row) * p.N + nb * BN + 32 * half;
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+              *reinterpret_cast<uint4 *>(dst + 4 * j) = make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host
+
+void tree_schedule(int n, uint8_t *merges);
+
+static int schedule_depth(int n, const uint8_t *merges) {
+  int depth = 0, maxd = 0;
+  for (int i = 0; i < n; i++) {
+    depth++;
+    maxd = std::max(maxd, depth);
+    depth -= merges[i];
+  }
+  return maxd;
+}
+
+static bi_status tree_check(const void *A, const void *W, int M, int N, int K, int shards) {
+  if (M < 0 || N <= 0 || K <= 0 || shards < 1) return BI_ERR_INVALID_ARG;
+  if (M > 0 && (!A || !W)) return BI_ERR_INVALID_ARG;
+  if (K % tg::LEAF != 0 || N % tg::BN != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int L = K / tg::LEAF;
+  if (!bi_pow2(shards) || L % shards != 0 || L / shards > tg::MAX_LEAVES) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(A) || !bi_aligned16(W)) return BI_ERR_UNSUPPORTED_SHAPE;
+  return BI_OK;
+}
+
+static bi_status tree_partials_launch(const void *A, const void *W, float *out, int M, int N, int K, int shards,
+                                      cudaStream_t stream) {
+  using namespace tg;
+  TreeGemmParams p{};
+  p.out = out;
+  p.status = status_word();
+  p.M = M; p.N = N; p.K = K; p.shards = shards;
+  p.leaves = K / LEAF / shards;
+  tree_schedule(p.leaves, p.merges);
+  if (schedule_depth(p.leaves, p.merges) > STACK_SLOTS + 1) return BI_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tmA, tmW;
+  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
+  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) != cudaSuccess)
+      return BI_ERR_CUDA;
+    attr_set = true;
+  }
+  const long tiles = (long)((M + BM - 1) / BM) * (N / BN) * shards;
+  const int grid = (int)std::min<long>(tiles, num_sms());
+  gemm_tree_kernel<<<grid, THREADS, SMEM, stream>>>(tmA, tmW, p);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace bi
+
+extern "C" size_t bi_gemm_tree_ws_bytes(int M, int N, int shards) {
+  if (M < 0 || N < 0 || shards <= 1) return 0;
+  return sizeof(float) * (size_t)shards * M * N;
+}
+
+extern "C" bi_status bi_gemm_tree_partials(const void *A, const void *W, float *partials, int M, int N, int K,
+                                           int shards, bi_stream_t stream) {
+  bi_status st = bi::tree_check(A, W, M, N, K, shards);
+  if (st != BI_OK) return st;
+  if (M > 0 && (!partials || !bi_aligned16(partials))) return partials ? BI_ERR_UNSUPPORTED_SHAPE : BI_ERR_INVALID_ARG;
+  if (M == 0) return BI_OK;
+  return bi::tree_partials_launch(A, W, partials, M, N, K, shards, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_gemm_tree(const void *A, const void *W, float *C, int M, int N, int K, int shards,
+                                  void *ws, size_t ws_bytes, bi_stream_t stream) {
+  bi_status st = bi::tree_check(A, W, M, N, K, shards);
+  if (st != BI_OK) return st;
+  if (M > 0 && !C) return BI_ERR_INVALID_ARG;
+  if (M > 0 && !bi_aligned16(C)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return BI_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (shards == 1) return bi::tree_partials_launch(A, W, C, M, N, K, 1, s);
+  const size_t need = bi_gemm_tree_ws_bytes(M, N, shards);
+  if (!ws || ws_bytes < need) return BI_ERR_WORKSPACE;
+  if (!bi_aligned16(ws)) return BI_ERR_UNSUPPORTED_SHAPE;
+  float *parts = static_cast<float *>(ws);
+  st = bi::tree_partials_launch(A, W, parts, M, N, K, shards, s);
+  if (st != BI_OK) return st;
+  return bi::tree_combine_launch(parts, C, shards, (size_t)M * N, s);
+}
