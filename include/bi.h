@@ -117,6 +117,28 @@ bi_status bi_lora_shrink_segmented(const void *x, const void *A, const void *pla
                                    int n_adapters, float *y, int M, int K, int r,
                                    int splits, int mode, bi_stream_t stream);
 
+/* Segmented shrink for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a convenience of this library.  Some
+ * callers cannot call cudaMalloc -- a plugin inside a host application that
+ * owns all device memory through its own pool and lets no library allocate,
+ * or a latency-critical loop where an allocation (which may synchronise the
+ * device) is not acceptable.  This call takes the adapter ids (int32 [M],
+ * device) instead of a plan and builds the plan in a fixed array of the
+ * library's own device memory: BI_NOALLOC_MAX_TOKENS + 258 int32 (about
+ * 257 KiB), held by every GPU that loads the library until the process exits.
+ * It allocates nothing.  Other arguments, results and guarantees are those of
+ * bi_lora_plan followed by bi_lora_shrink_segmented (same bits).
+ * M > BI_NOALLOC_MAX_TOKENS or n_adapters > 256 returns
+ * BI_ERR_UNSUPPORTED_SHAPE before any work.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress) and caches it; make
+ * that first call before any stream capture.  All calls share the one array,
+ * so calls whose kernels overlap on the GPU (different streams or threads)
+ * race on it and must be serialised by the caller. */
+#define BI_NOALLOC_MAX_TOKENS 65536
+bi_status bi_lora_shrink_segmented_noalloc(const void *x, const void *A, const int32_t *ids,
+                                           int n_adapters, float *y, int M, int K, int r,
+                                           int splits, int mode, bi_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* LoRA expand [LoRA Q&A: the second low-rank product]:                 */
 /*   e[t][n] = sum_j bf16(y[t][j]) * B[n][j]                            */

@@ -38,6 +38,7 @@ _SIGS = {
     "bi_lora_plan_bytes": (Z, [I, I]),
     "bi_lora_plan": (I, [P, I, I, P, Z, P]),
     "bi_lora_shrink_segmented": (I, [P, P, P, I, P, I, I, I, I, I, P]),
+    "bi_lora_shrink_segmented_noalloc": (I, [P, P, P, I, P, I, I, I, I, I, P]),
     "bi_lora_expand": (I, [P, P, P, I, I, I, I, P]),
     "bi_lora_expand_segmented": (I, [P, P, P, I, P, I, I, I, I, P]),
     "bi_gemm": (I, [P, P, P, I, I, I, I, P]),
@@ -146,6 +147,27 @@ def lora_shrink_segmented(x, A, plan, y, splits=8, mode="tree", stream=None):
     if plan.numel() * 4 < lora_plan_bytes(M, n_ad):
         raise ValueError("plan too small")
     _call("bi_lora_shrink_segmented", _ptr(x), _ptr(A), _ptr(plan), n_ad, _ptr(y), M, K, r,
+          splits, MODES[mode], _stream(stream))
+    return y
+
+
+NOALLOC_MAX_TOKENS = 65536
+
+
+def lora_shrink_segmented_noalloc(x, A, ids, y, splits=8, mode="tree", stream=None):
+    """Segmented shrink that allocates nothing: ids int32 [M] go straight to
+    the library, which builds the token plan in its own fixed device array
+    (M <= NOALLOC_MAX_TOKENS).  Calls that overlap on the GPU race on that
+    array; serialise them."""
+    _check(x, "x", torch.bfloat16, 2)
+    _check(A, "A", torch.bfloat16, 3)
+    _check(ids, "ids", torch.int32, 1)
+    _check(y, "y", torch.float32, 2)
+    M, K = x.shape
+    n_ad, r, K2 = A.shape
+    if K2 != K or tuple(y.shape) != (M, r) or ids.shape[0] != M:
+        raise ValueError("shape mismatch")
+    _call("bi_lora_shrink_segmented_noalloc", _ptr(x), _ptr(A), _ptr(ids), n_ad, _ptr(y), M, K, r,
           splits, MODES[mode], _stream(stream))
     return y
 
