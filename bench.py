@@ -221,62 +221,103 @@ class Workload:
         return out
 
 
+KERNEL_REPS = 10      # reps per kernel graph in the per-kernel timing block
+
+
+def capture(fn, stream):
+    """Capture fn() into a CUDA graph on `stream`."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
 def run_ours(args, rank, world, device):
     from invariant_bi_lora_b200 import bi, synth
     wl = Workload(bi, synth, seed=0)
-    stream = torch.cuda.current_stream()
     pk = peaks()
+    cs = torch.cuda.Stream()                       # capture / launch stream
 
-    def step(events=None):
+    def step_body():
         for i, (name, fn, *_rest) in enumerate(wl.kernels):
             wl.flush.fill_(i & 0xff)               # L2 flush: 256 MiB write
-            if events is not None:
-                events[i][0].record(stream)
             fn()
-            if events is not None:
-                events[i][1].record(stream)
 
-    clocks = ClockSampler(device)
-    clocks.start()
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if bi.get_device_status() != 0:
-        raise RuntimeError("device status set during warm-up")
+    # everything below runs with cs as the current stream: graph replays go to
+    # the current stream, and the timing events must be on the same one
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        # eager warm-up (TMA descriptors, kernel attributes, occupancy queries)
+        for _ in range(args.warmup):
+            step_body()
+        torch.cuda.synchronize()
+        if bi.get_device_status(cs) != 0:
+            raise RuntimeError("device status set during warm-up")
 
-    nk = len(wl.kernels)
-    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
-          for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # one step = one replay of this graph: every kernel once, each after a flush
+        g_step = capture(step_body, cs)
+        # per-kernel graphs for the difference timing: R x (flush, kernel) and R x flush
+        R = KERNEL_REPS
+        def reps(fn):
+            def body():
+                for i in range(R):
+                    wl.flush.fill_(i & 0xff)
+                    if fn is not None:
+                        fn()
+            return body
+        g_flush = capture(reps(None), cs)
+        g_kern = [capture(reps(fn), cs) for (name, fn, *_r) in wl.kernels]
+        for _ in range(args.warmup):
+            g_step.replay()
+        torch.cuda.synchronize()
+
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(device)
+        clocks.start()
+        time.sleep(0.3)
+        # ---------------- timed region: exactly K steps
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        h0 = time.time()
+        t0, t1 = ev(), ev()
+        t0.record(cs)
+        for _ in range(args.steps):
+            g_step.replay()
+        t1.record(cs)
+        torch.cuda.synchronize()
+        h1 = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        clocks.mark(h0, h1)
+        total_ms = t0.elapsed_time(t1)
+
+        # ---------------- per-kernel durations: (R x [flush, kernel]) - (R x [flush])
+        per = {name: [] for (name, *_r) in wl.kernels}
+        for _ in range(3):
+            a, b = ev(), ev()
+            a.record(cs); g_flush.replay(); b.record(cs)
+            torch.cuda.synchronize()
+            tf = a.elapsed_time(b)
+            for (name, *_r), g in zip(wl.kernels, g_kern):
+                a, b = ev(), ev()
+                a.record(cs); g.replay(); b.record(cs)
+                torch.cuda.synchronize()
+                per[name].append(max(a.elapsed_time(b) - tf, 1e-6) / R)
+        clk = clocks.stop()
+    for k, v in per.items():
+        sys.stderr.write(f"kernel {k}: {[round(t * 1e3, 2) for t in v]} us\n")
+    per = {k: statistics.median(v) for k, v in per.items()}
     if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    h0 = time.time()
-    t0.record(stream)
-    for s in range(args.steps):
-        step(ev[s])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    h1 = time.time()
-    if world > 1:
-        torch.distributed.barrier()
-    clocks.mark(h0, h1)
-    clk = clocks.stop()
-    total_ms = t0.elapsed_time(t1)
-    per = {name: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
-           for i, (name, *_r) in enumerate(wl.kernels)}
-    if world > 1:
-        t = torch.tensor([total_ms] + [sum(v) for v in per.values()], device="cuda")
+        t = torch.tensor([total_ms] + list(per.values()), device="cuda")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t[0])
-        for j, k in enumerate(per):
-            scale = float(t[j + 1]) / max(sum(per[k]), 1e-9)
-            per[k] = [v * scale for v in per[k]]
-    status = bi.get_device_status()
+        per = {k: float(t[j + 1]) for j, k in enumerate(per)}
+    status = bi.get_device_status(cs)
 
     kern = []
     for (name, fn, nbytes, flops, bound, launches) in wl.kernels:
-        ms = statistics.mean(per[name])
+        ms = per[name]
         gbs = nbytes / (ms * 1e-3) / 1e9
         tfl = flops / (ms * 1e-3) / 1e12 if flops else None
         if bound == "tensor":
@@ -293,6 +334,7 @@ def run_ours(args, rank, world, device):
     value = world * tree["gbs"]
     gemm = by.get("gemm")
     e2e = measure_e2e(wl, bi, args) if rank == 0 else None
+    atomic_var = atomic_variation(wl, bi) if rank == 0 else None
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -301,7 +343,9 @@ def run_ours(args, rank, world, device):
         "data": "synthetic (seeded numpy PCG64; shapes of the pages' workloads)",
         "config": {"workload": WORKLOAD, "global_batch": M4 * world, "seq_len": None,
                    "parallelism": f"dp{world} (independent replicas, no collective)",
-                   "l2": "flushed before every kernel (256 MiB write)"},
+                   "l2": "flushed before every kernel (256 MiB write)",
+                   "timing": "step = one CUDA-graph replay of the whole path; per-kernel time = "
+                             f"(graph of {R} x [flush, kernel]) - (graph of {R} x [flush]), CUDA events"},
         "roofline": {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"],
                      "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
                      "traffic": None, "peak_source": pk["source"]},
@@ -310,13 +354,39 @@ def run_ours(args, rank, world, device):
         "delta_vs_atomic_pct": round(100.0 * (tree["us"] / by["shrink_atomic_s8"]["us"] - 1.0), 2),
         "speedup_vs_unsplit_pct": round(100.0 * (by["shrink_unsplit"]["us"] / tree["us"] - 1.0), 2),
         "bi_gemm_tflops": None if gemm is None else gemm["tflops"],
+        "atomic_variation": atomic_var,
         "kernels": kern,
+        "kernel_sum_ms": round(sum(per.values()), 4),
         "gpu_launches": args.steps * sum(k["launches"] for k in kern),
         "device_status": status,
         "clocks": clk,
         "e2e": e2e,
     }
     return line
+
+
+def atomic_variation(wl, bi, replays=100):
+    """Identical-input replays of the M=16 shrink (split-K 8): the fraction
+    of replay pairs whose outputs differ anywhere and the fraction of
+    elements that differ from replay 0, for the atomic and the tree mode.
+    Outside the timed region."""
+    out = {}
+    for mode in ("atomic", "tree"):
+        outs = []
+        for _ in range(replays):
+            bi.lora_shrink(wl.x16, wl.A16, wl.y16, 8, mode)
+            outs.append(wl.y16.clone())
+        torch.cuda.synchronize()
+        h = torch.stack(outs).view(torch.int32).cpu().numpy().reshape(replays, -1)
+        uniq = len({row.tobytes() for row in h})
+        pairs_diff = 0
+        for i in range(replays):
+            pairs_diff += int(np.sum(np.any(h[i + 1:] != h[i], axis=1)))
+        npairs = replays * (replays - 1) // 2
+        out[mode] = {"replays": replays, "distinct_outputs": uniq,
+                     "pairs_differing": round(pairs_diff / npairs, 4),
+                     "elements_differing_vs_first": round(float(np.mean(h[1:] != h[0])), 4)}
+    return out
 
 
 def measure_e2e(wl, bi, args):

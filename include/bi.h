@@ -212,7 +212,7 @@ bi_status bi_tree_combine(const float *partials, float *out, int s, size_t count
 bi_status bi_rmsnorm(const void *x, const void *w, void *y, int rows, int n,
                      float eps, bi_stream_t stream);
 
-/* log_softmax [BIO]: T = 1024, V = 4.  m = row max; d = x - m;
+/* log_softmax [BIO]: T = 4096, V = 4.  m = row max; d = x - m;
  * S = canonical sum of bi_exp(d); L = bi_log(S); out = fl(d - L).
  * bi_exp / bi_log are the library's own written methods (Cody-Waite +
  * Taylor; atanh series), bitwise reproducible on any IEEE machine.
@@ -225,7 +225,9 @@ bi_status bi_mean(const float *x, float *out, int rows, int n, bi_stream_t strea
 
 /* The library's exp (which = 0) or log (which = 1) of bi_log_softmax,
  * applied elementwise: y[i] = bi_exp(x[i]) or bi_log(x[i]).  x, y fp32 [n].
- * bi_log is defined for positive normal x; bi_exp for x <= 88. */
+ * bi_log is defined for positive normal x; bi_exp for x <= 88.  which = 2
+ * runs the shortcut of bi_exp that log_softmax takes for -87 <= x <= 88
+ * (same bits as bi_exp there; undefined outside). */
 bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream);
 
 /* ------------------------------------------------------------------ */

@@ -296,10 +296,12 @@ def mean(x, out, stream=None):
 
 
 def math_spec(x, y, which, stream=None):
-    """y = the library's exp (which='exp') or log (which='log') of x."""
+    """y = the library's exp (which='exp'), log ('log') or the exp shortcut
+    log_softmax uses on [-87, 88] ('exp_fast') of x."""
     _check(x, "x", torch.float32)
     _check(y, "y", torch.float32)
-    _call("bi_math_spec", _ptr(x), _ptr(y), x.numel(), {"exp": 0, "log": 1}[which], _stream(stream))
+    _call("bi_math_spec", _ptr(x), _ptr(y), x.numel(), {"exp": 0, "log": 1, "exp_fast": 2}[which],
+          _stream(stream))
     return y
 
 

@@ -48,6 +48,32 @@ BI_DEV float bi_exp(float x) {
   return __fmul_rn(p, pow2_exact(ni));
 }
 
+// bi_exp for -87 <= x <= 88: the same operations and the same bits as
+// bi_exp there, with the rounding to an integer done by adding and
+// subtracting 1.5 * 2^23 (nearest, ties to even -- what rint does for
+// |t| < 2^22) and the integer read from the sum's low bits; the scale 2^n is
+// a normal number over the whole range, so the result is one multiply.
+BI_DEV float bi_exp_fast(float x) {
+  const float log2e = (float)1.4426950408889634074;
+  const float ln2_head = 0.693145751953125f;
+  const float ln2_tail = (float)(0.693147180559945309417 - 0.693145751953125);
+  const float magic = 12582912.0f;                    // 1.5 * 2^23
+  const float sh = __fadd_rn(__fmul_rn(x, log2e), magic);
+  const float n = __fsub_rn(sh, magic);
+  const int ni = __float_as_int(sh) - __float_as_int(magic);
+  float r = __fmaf_rn(-n, ln2_head, x);
+  r = __fmaf_rn(-n, ln2_tail, r);
+  float p = (float)(1.0 / 5040.0);
+  p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+}
+
 BI_DEV float bi_log(float x) {
   const float ln2_head = 0.693145751953125f;
   const float ln2_tail = (float)(0.693147180559945309417 - 0.693145751953125);

@@ -10,7 +10,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/bi.h"
+#include "bi.h"
 
 #define BI_DEV __device__ __forceinline__
 

@@ -75,40 +75,51 @@ expand_kernel(const __grid_constant__ ExpandParams p) {
   }
 
   const uint16_t *bad = p.bt + (size_t)ti.adapter * p.N * p.r;
-#pragma unroll 2
-  for (int nt = 0; nt < 8; nt++) {
-    const int n0 = nbase + nt * 8;
-    if (n0 >= p.N) break;
-    const uint16_t *brow = bad + (size_t)(n0 + g) * p.r;   // B[n0+g][.]
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // B fragments of NB n-tiles at a time first (independent L2 loads in
+  // flight together), then their MMAs and stores
+  constexpr int NB = KS <= 2 ? 8 : (KS <= 4 ? 4 : 2);
+#pragma unroll 1
+  for (int nb0 = 0; nb0 < 8; nb0 += NB) {
+    uint32_t bfr[NB][KS][2];
 #pragma unroll
-    for (int s = 0; s < KS; s++) {
-      const int k0 = 16 * s + 2 * c, k1 = k0 + 8;
-      uint32_t b[2];
-      b[0] = k0 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k0)) : 0u;
-      b[1] = k1 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k1)) : 0u;
-      mma_bf16_16816(acc, afr[s], b, acc);
-    }
-    const int n = n0 + 2 * c;
-    if (v0) {
-      float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row0 * p.N + n);
-      float2 v = make_float2(acc[0], acc[1]);
-      if (p.accumulate) {
-        const float2 q = *o;
-        v.x = __fadd_rn(q.x, v.x);
-        v.y = __fadd_rn(q.y, v.y);
+    for (int i = 0; i < NB; i++) {
+      const int n0 = nbase + (nb0 + i) * 8;
+      const uint16_t *brow = bad + (size_t)(n0 + g) * p.r;   // B[n0+g][.]
+      const bool ok = n0 < p.N;
+#pragma unroll
+      for (int s = 0; s < KS; s++) {
+        const int k0 = 16 * s + 2 * c, k1 = k0 + 8;
+        bfr[i][s][0] = ok && k0 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k0)) : 0u;
+        bfr[i][s][1] = ok && k1 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k1)) : 0u;
       }
-      *o = v;
     }
-    if (v1) {
-      float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row1 * p.N + n);
-      float2 v = make_float2(acc[2], acc[3]);
-      if (p.accumulate) {
-        const float2 q = *o;
-        v.x = __fadd_rn(q.x, v.x);
-        v.y = __fadd_rn(q.y, v.y);
+#pragma unroll
+    for (int i = 0; i < NB; i++) {
+      const int n0 = nbase + (nb0 + i) * 8;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < KS; s++) mma_bf16_16816(acc, afr[s], bfr[i][s], acc);
+      const int n = n0 + 2 * c;
+      if (v0 && n0 < p.N) {
+        float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row0 * p.N + n);
+        float2 v = make_float2(acc[0], acc[1]);
+        if (p.accumulate) {
+          const float2 q = *o;
+          v.x = __fadd_rn(q.x, v.x);
+          v.y = __fadd_rn(q.y, v.y);
+        }
+        __stcs(o, v);
       }
-      *o = v;
+      if (v1 && n0 < p.N) {
+        float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row1 * p.N + n);
+        float2 v = make_float2(acc[2], acc[3]);
+        if (p.accumulate) {
+          const float2 q = *o;
+          v.x = __fadd_rn(q.x, v.x);
+          v.y = __fadd_rn(q.y, v.y);
+        }
+        __stcs(o, v);
+      }
     }
   }
 }

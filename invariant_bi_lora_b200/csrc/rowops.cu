@@ -13,6 +13,7 @@
 // (which is that tree), across warps and CTAs by perfect trees over
 // power-of-two counts.  Vectors are 16 bytes: V = 8 for bf16, V = 4 for fp32.
 #include "bimath.cuh"
+#include "tc.cuh"
 
 #include <cooperative_groups.h>
 #include <algorithm>
@@ -22,47 +23,66 @@ namespace cg = cooperative_groups;
 namespace bi {
 
 // ======================================================================
-// RMSNorm: T = 512 lanes of V = 8 bf16; one CTA of 512 threads per row,
-// thread t = lane t.  The row stays in registers (VPL vectors per lane)
-// between the sum and the scaling, so x is read from HBM once.
+// RMSNorm: T = 512 lanes of V = 8 bf16.  One CTA of THREADS threads per
+// row; thread u owns the LPT = 512/THREADS adjacent lanes u*LPT .. +LPT-1
+// (a subtree of the lane tree), so it reads LPT*16 contiguous bytes per
+// step.  The row stays in registers (VPL vectors per lane) between the sum
+// and the scaling, so x is read from HBM once.  128 threads per row keep 16
+// rows (128 KB) in flight per SM.
 // ======================================================================
 constexpr int kNormT = 512;
 
-template <int VPL>
-__global__ void __launch_bounds__(kNormT)
+template <int THREADS, int VPL>
+__global__ void __launch_bounds__(THREADS)
 rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
                uint16_t *__restrict__ y, int n, float eps) {
-  __shared__ float s_warp[kNormT / 32];
+  constexpr int LPT = kNormT / THREADS;
+  constexpr int NW = THREADS / 32;
+  __shared__ float s_warp[NW];
   __shared__ float s_inv;
-  const int t = threadIdx.x;
+  const int u = threadIdx.x;
   const size_t row = blockIdx.x;
   const int nvec = n / 8;
   const uint16_t *xr = x + row * n;
 
-  uint4 v[VPL];
-  float p = 0.0f;
+  uint4 v[VPL][LPT];
+  float p[LPT];
 #pragma unroll
-  for (int j = 0; j < VPL; j++) {
-    const int vi = t + j * kNormT;
-    if (vi < nvec) {
-      v[j] = ldg128_stream(xr + 8 * vi);
-      const uint32_t q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+  for (int l = 0; l < LPT; l++) p[l] = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 4; e++) {
-        const float a = bf16lo(q[e]), b = bf16hi(q[e]);
-        p = __fadd_rn(p, __fmul_rn(a, a));
-        p = __fadd_rn(p, __fmul_rn(b, b));
+  for (int j = 0; j < VPL; j++)
+#pragma unroll
+    for (int l = 0; l < LPT; l++) {
+      const int vi = j * kNormT + u * LPT + l;
+      v[j][l] = vi < nvec ? ldg128_stream(xr + 8 * vi) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+  for (int j = 0; j < VPL; j++)
+#pragma unroll
+    for (int l = 0; l < LPT; l++) {
+      if (j * kNormT + u * LPT + l < nvec) {
+        const uint32_t q[4] = {v[j][l].x, v[j][l].y, v[j][l].z, v[j][l].w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const float a = bf16lo(q[e]), b = bf16hi(q[e]);
+          p[l] = __fadd_rn(p[l], __fmul_rn(a, a));
+          p[l] = __fadd_rn(p[l], __fmul_rn(b, b));
+        }
       }
     }
-  }
-  p = warp_tree_sum(p);
-  if ((t & 31) == 0) s_warp[t >> 5] = p;
-  __syncthreads();
-  if (t < 32) {
-    float q = t < kNormT / 32 ? s_warp[t] : 0.0f;
+  // perfect tree over this thread's LPT adjacent lanes
 #pragma unroll
-    for (int o = 1; o < kNormT / 32; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
-    if (t == 0) {
+  for (int st = 1; st < LPT; st <<= 1)
+#pragma unroll
+    for (int l = 0; l + st < LPT; l += 2 * st) p[l] = __fadd_rn(p[l], p[l + st]);
+  float sum = warp_tree_sum(p[0]);
+  if ((u & 31) == 0) s_warp[u >> 5] = sum;
+  __syncthreads();
+  if (u < 32) {
+    float q = u < NW ? s_warp[u] : 0.0f;
+#pragma unroll
+    for (int o = 1; o < NW; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+    if (u == 0) {
       const float ms = __fdiv_rn(q, (float)n);
       s_inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
     }
@@ -71,22 +91,24 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
   const float inv = s_inv;
   uint16_t *yr = y + row * n;
 #pragma unroll
-  for (int j = 0; j < VPL; j++) {
-    const int vi = t + j * kNormT;
-    if (vi < nvec) {
-      const uint4 wv = ldg128(w + 8 * vi);
-      const uint32_t q[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-      const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
-      uint32_t o[4];
+  for (int j = 0; j < VPL; j++)
 #pragma unroll
-      for (int e = 0; e < 4; e++) {
-        const float lo = __fmul_rn(__fmul_rn(bf16lo(q[e]), inv), bf16lo(wq[e]));
-        const float hi = __fmul_rn(__fmul_rn(bf16hi(q[e]), inv), bf16hi(wq[e]));
-        o[e] = pack_bf16x2(lo, hi);
+    for (int l = 0; l < LPT; l++) {
+      const int vi = j * kNormT + u * LPT + l;
+      if (vi < nvec) {
+        const uint4 wv = ldg128(w + 8 * vi);
+        const uint32_t q[4] = {v[j][l].x, v[j][l].y, v[j][l].z, v[j][l].w};
+        const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const float lo = __fmul_rn(__fmul_rn(bf16lo(q[e]), inv), bf16lo(wq[e]));
+          const float hi = __fmul_rn(__fmul_rn(bf16hi(q[e]), inv), bf16hi(wq[e]));
+          o[e] = pack_bf16x2(lo, hi);
+        }
+        *reinterpret_cast<uint4 *>(yr + 8 * vi) = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      *reinterpret_cast<uint4 *>(yr + 8 * vi) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-  }
 }
 
 // ======================================================================
@@ -135,31 +157,53 @@ mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
 }
 
 // ======================================================================
-// log_softmax: T = 1024 lanes of V = 4 fp32, two passes over the row
+// log_softmax: T = 4096 lanes of V = 4 fp32, two passes over the row
 // (max; then the canonical sum of bi_exp(x - max)), then the write.  The
 // row is held on chip between the passes so HBM sees one read and one
 // write: a cluster of C CTAs shares the row, CTA q owning lanes
-// [q*1024/C, (q+1)*1024/C) -- a subtree of the lane tree -- and keeping
-// its lanes' vectors in shared memory (slot [j][tau] for vector
-// 1024*j + lane).  Maxima and sums meet through distributed shared memory.
+// [q*4096/C, (q+1)*4096/C) -- a subtree of the lane tree -- one thread per
+// lane, each keeping its lane's vectors in shared memory (slot [j][tau] for
+// vector 4096*j + lane).  Maxima and sums meet through distributed shared
+// memory.  The sum pass stores d = x - max back into the slot, so the write
+// pass is one subtraction per element.
 // ======================================================================
+constexpr int kLsmT = 4096;
+
 struct LsmParams {
   const float *x;
   float *out;
+  unsigned *status;
   int n;
-  int C;      // CTAs per row (cluster size), power of two
-  int J;      // vector slots per lane = ceil(n/4 / 1024)
+  int C;      // CTAs per row (cluster size), power of two, 4..16
+  int J;      // vector slots per lane = ceil(n/4 / 4096)
 };
+
+BI_DEV float4 bi_exp4(float4 d) {
+  float4 e;
+  if (fminf(fminf(d.x, d.y), fminf(d.z, d.w)) >= -87.0f) {
+    e.x = bi_exp_fast(d.x);
+    e.y = bi_exp_fast(d.y);
+    e.z = bi_exp_fast(d.z);
+    e.w = bi_exp_fast(d.w);
+  } else {
+    e.x = bi_exp(d.x);
+    e.y = bi_exp(d.y);
+    e.z = bi_exp(d.z);
+    e.w = bi_exp(d.w);
+  }
+  return e;
+}
 
 __global__ void __launch_bounds__(1024)
 log_softmax_kernel(const __grid_constant__ LsmParams p) {
   extern __shared__ float4 lsm_smem[];
   __shared__ float s_red[32];
   __shared__ float s_max, s_sum;
+  __shared__ __align__(8) uint64_t s_bar;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C;
   const int q = (int)cluster.block_rank();
-  const int lpc = kLaneT / C;                  // lanes (= threads) per CTA
+  const int lpc = kLsmT / C;                   // lanes (= threads) per CTA
   const int tau = threadIdx.x;
   const int lane_id = q * lpc + tau;           // logical lane
   const size_t row = blockIdx.x / C;
@@ -167,16 +211,26 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   const float4 *xr = reinterpret_cast<const float4 *>(p.x + row * p.n);
   float4 *outr = reinterpret_cast<float4 *>(p.out + row * p.n);
   const int nwarps = lpc / 32;
+  // this lane's vectors: 4096*j + lane_id for j < nj
+  const int nj = lane_id < nvec ? (nvec - 1 - lane_id) / kLsmT + 1 : 0;
 
-  // ---- load this lane's vectors into its shared-memory slots; local max
+  // ---- this lane's vectors -> its shared-memory slots: 16-byte cp.async
+  // copies, all in flight at once; each thread's arrival on the barrier
+  // fires when its copies have landed.
+  if (tau == 0) {
+    mbar_init(&s_bar, blockDim.x);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  for (int j = 0; j < nj; j++) cp_async16(lsm_smem + (size_t)j * lpc + tau, xr + (size_t)j * kLsmT + lane_id);
+  cp_async_arrive(&s_bar);
+  if (!mbar_wait(&s_bar, 0)) flag_error(p.status, BI_ERR_TIMEOUT);
+
+  // ---- local max
   float m = -INFINITY;
-  for (int j = 0; j < p.J; j++) {
-    const int vi = j * kLaneT + lane_id;
-    if (vi < nvec) {
-      const float4 v = __ldcs(xr + vi);
-      lsm_smem[j * lpc + tau] = v;
-      m = fmaxf(fmaxf(m, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
-    }
+  for (int j = 0; j < nj; j++) {
+    const float4 v = lsm_smem[j * lpc + tau];
+    m = fmaxf(fmaxf(m, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
   }
   m = warp_max(m);
   if ((tau & 31) == 0) s_red[tau >> 5] = m;
@@ -191,17 +245,21 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   float rmax = -INFINITY;
   for (int r = 0; r < C; r++) rmax = fmaxf(rmax, *cluster.map_shared_rank(&s_max, r));
 
-  // ---- lane chain of bi_exp(x - max)
+  // ---- lane chain of bi_exp(x - max); d = x - max stays in the slot
   float s = 0.0f;
-  for (int j = 0; j < p.J; j++) {
-    const int vi = j * kLaneT + lane_id;
-    if (vi < nvec) {
-      const float4 v = lsm_smem[j * lpc + tau];
-      s = __fadd_rn(s, bi_exp(__fsub_rn(v.x, rmax)));
-      s = __fadd_rn(s, bi_exp(__fsub_rn(v.y, rmax)));
-      s = __fadd_rn(s, bi_exp(__fsub_rn(v.z, rmax)));
-      s = __fadd_rn(s, bi_exp(__fsub_rn(v.w, rmax)));
-    }
+#pragma unroll 2
+  for (int j = 0; j < nj; j++) {
+    float4 d = lsm_smem[j * lpc + tau];
+    d.x = __fsub_rn(d.x, rmax);
+    d.y = __fsub_rn(d.y, rmax);
+    d.z = __fsub_rn(d.z, rmax);
+    d.w = __fsub_rn(d.w, rmax);
+    lsm_smem[j * lpc + tau] = d;
+    const float4 e = bi_exp4(d);
+    s = __fadd_rn(s, e.x);
+    s = __fadd_rn(s, e.y);
+    s = __fadd_rn(s, e.z);
+    s = __fadd_rn(s, e.w);
   }
   s = warp_tree_sum(s);
   __syncthreads();                      // s_red reuse
@@ -224,18 +282,15 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
       if (r + st < C) part[r] = __fadd_rn(part[r], part[r + st]);
   const float L = bi_log(part[0]);
 
-  // ---- write out = (x - max) - L
-  for (int j = 0; j < p.J; j++) {
-    const int vi = j * kLaneT + lane_id;
-    if (vi < nvec) {
-      const float4 v = lsm_smem[j * lpc + tau];
-      float4 o;
-      o.x = __fsub_rn(__fsub_rn(v.x, rmax), L);
-      o.y = __fsub_rn(__fsub_rn(v.y, rmax), L);
-      o.z = __fsub_rn(__fsub_rn(v.z, rmax), L);
-      o.w = __fsub_rn(__fsub_rn(v.w, rmax), L);
-      __stcs(outr + vi, o);
-    }
+  // ---- write out = d - L
+  for (int j = 0; j < nj; j++) {
+    const float4 d = lsm_smem[j * lpc + tau];
+    float4 o;
+    o.x = __fsub_rn(d.x, L);
+    o.y = __fsub_rn(d.y, L);
+    o.z = __fsub_rn(d.z, L);
+    o.w = __fsub_rn(d.w, L);
+    __stcs(outr + (size_t)j * kLsmT + lane_id, o);
   }
   cluster.sync();   // peers may still read s_max / s_sum of this CTA
 }
@@ -245,7 +300,7 @@ __global__ void math_spec_kernel(const float *__restrict__ x, float *__restrict_
                                  int which) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
-    y[i] = which == 0 ? bi_exp(x[i]) : bi_log(x[i]);
+    y[i] = which == 0 ? bi_exp(x[i]) : (which == 1 ? bi_log(x[i]) : bi_exp_fast(x[i]));
 }
 
 }  // namespace bi
@@ -263,10 +318,12 @@ extern "C" bi_status bi_rmsnorm(const void *x, const void *w, void *y, int rows,
   auto xp = static_cast<const uint16_t *>(x);
   auto wp = static_cast<const uint16_t *>(w);
   auto yp = static_cast<uint16_t *>(y);
-  if (vpl <= 1) bi::rmsnorm_kernel<1><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
-  else if (vpl <= 2) bi::rmsnorm_kernel<2><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
-  else if (vpl <= 4) bi::rmsnorm_kernel<4><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
-  else bi::rmsnorm_kernel<8><<<rows, bi::kNormT, 0, s>>>(xp, wp, yp, n, eps);
+  // thread count per row is bit-neutral (lanes are logical); 128 threads
+  // with 4 lanes each while the row fits in registers
+  if (vpl <= 1) bi::rmsnorm_kernel<128, 1><<<rows, 128, 0, s>>>(xp, wp, yp, n, eps);
+  else if (vpl <= 2) bi::rmsnorm_kernel<128, 2><<<rows, 128, 0, s>>>(xp, wp, yp, n, eps);
+  else if (vpl <= 4) bi::rmsnorm_kernel<128, 4><<<rows, 128, 0, s>>>(xp, wp, yp, n, eps);
+  else bi::rmsnorm_kernel<256, 8><<<rows, 256, 0, s>>>(xp, wp, yp, n, eps);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
@@ -286,15 +343,15 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
   if (n % 4 != 0 || n > 262144) return BI_ERR_UNSUPPORTED_SHAPE;
   if (!bi_aligned16(x) || !bi_aligned16(out)) return BI_ERR_UNSUPPORTED_SHAPE;
   if (rows == 0) return BI_OK;
-  bi::LsmParams p{x, out, n, 1, 0};
+  bi::LsmParams p{x, out, bi::status_word(), n, 4, 0};
   const int nvec = n / 4;
-  p.J = (nvec + bi::kLaneT - 1) / bi::kLaneT;
-  // Smallest cluster whose per-CTA share of the row fits in ~80 KB of
-  // shared memory (two CTAs per SM), at most 16.  Bit-neutral.
-  int C = 1;
-  while (C < 16 && (size_t)p.J * (bi::kLaneT / C) * 16 > 80 * 1024) C *= 2;
+  p.J = (nvec + bi::kLsmT - 1) / bi::kLsmT;
+  // Smallest cluster (4..16 CTAs, at most 1024 threads each) whose share of
+  // the row fits in ~80 KB of shared memory, two CTAs per SM.  Bit-neutral.
+  int C = 4;
+  while (C < 16 && (size_t)p.J * (bi::kLsmT / C) * 16 > 80 * 1024) C *= 2;
   p.C = C;
-  const size_t smem = (size_t)p.J * (bi::kLaneT / C) * 16;
+  const size_t smem = (size_t)p.J * (bi::kLsmT / C) * 16;
   if (smem > 200 * 1024) return BI_ERR_UNSUPPORTED_SHAPE;
   cudaError_t e = cudaFuncSetAttribute(bi::log_softmax_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -305,7 +362,7 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)rows * C, 1, 1);
-  cfg.blockDim = dim3(bi::kLaneT / C, 1, 1);
+  cfg.blockDim = dim3(bi::kLsmT / C, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
@@ -320,7 +377,7 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
 }
 
 extern "C" bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream) {
-  if ((n > 0 && (!x || !y)) || (which != 0 && which != 1)) return BI_ERR_INVALID_ARG;
+  if ((n > 0 && (!x || !y)) || which < 0 || which > 2) return BI_ERR_INVALID_ARG;
   if (n == 0) return BI_OK;
   const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16);
   bi::math_spec_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, which);

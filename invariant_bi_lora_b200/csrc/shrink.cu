@@ -27,8 +27,10 @@
 // (g, c) feeds k = 8c..8c+7 to MMA k-slots {2c, 2c+1, 2c+8, 2c+9} of two
 // MMAs; the same permutation is applied to both operands, so the products
 // summed are exactly x[m][k] * A[j][k].  No shared-memory staging: the loads
-// go straight to registers, one leaf ahead of the MMAs.
-#include "common.cuh"
+// go straight to registers through a ring of PF leaves per warp, so every
+// warp keeps PF leaves of loads in flight while it multiplies -- the kernel
+// is HBM-bound, and the ring depth is what hides DRAM latency.
+#include "tc.cuh"
 
 #include <cooperative_groups.h>
 #include <algorithm>
@@ -57,6 +59,9 @@ struct ShrinkParams {
   int mtiles;               // MT: 16-row MMA tiles per CTA
   int ngroups;              // NG: rank groups of NGW columns
   int mode;
+  int a_staged;             // 1: the CTA's A slice sits in shared memory
+  int a_offset;             // bytes from the start of dynamic shared memory to the A slice
+  int ring_offset;          // bytes from the start of dynamic shared memory to the warp rings
   uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
 };
 
@@ -67,19 +72,6 @@ struct LeafFrag {
   uint4 xa[2][2];     // [chunk][row g / row g+8]
   uint4 ab[2][NT];    // [chunk][n-tile]
 };
-
-template <int NT>
-BI_DEV void load_leaf(LeafFrag<NT> &f, const uint16_t *xr0, const uint16_t *xr1, bool v0,
-                      bool v1, const uint16_t *const *acol, int k) {
-#pragma unroll
-  for (int h = 0; h < 2; h++) {
-    const int kk = k + 32 * h;
-    f.xa[h][0] = v0 ? ldg128_stream(xr0 + kk) : make_uint4(0, 0, 0, 0);
-    f.xa[h][1] = v1 ? ldg128_stream(xr1 + kk) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int t = 0; t < NT; t++) f.ab[h][t] = ldg128(acol[t] + kk);
-  }
-}
 
 // One leaf: four MMAs per n-tile (two k chunks x two k16 steps), from zero.
 template <int NT>
@@ -104,7 +96,7 @@ BI_DEV void mma_leaf(float acc[NT][4], const LeafFrag<NT> &f) {
   }
 }
 
-template <int NGW, int MAXD>
+template <int NGW, int MAXD, int PF>
 __global__ void __launch_bounds__(256)
 shrink_kernel(const __grid_constant__ ShrinkParams p) {
   constexpr int NT = NGW / 8;
@@ -141,15 +133,58 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   // rows g and g+8 of this warp's m-tile
   const int lr0 = mt * 16 + g, lr1 = lr0 + 8;       // local rows in the tile
   const bool v0 = lr0 < ti.rows, v1 = lr1 < ti.rows;
-  int row0 = 0, row1 = 0;
-  if (v0) row0 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr0] : ti.row0 + lr0;
-  if (v1) row1 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr1] : ti.row0 + lr1;
-  const uint16_t *xr0 = p.x + (size_t)row0 * p.K + 8 * c;
-  const uint16_t *xr1 = p.x + (size_t)row1 * p.K + 8 * c;
-  const uint16_t *acol[NT];
+
+  // ---- shared memory: the CTA's A slice (staged once when it fits) and a
+  // per-warp ring of PF leaf slots.  Rows are 128 bytes per leaf; the
+  // 16-byte chunk index is XOR-ed with (row & 1) << 2 so that the two rows a
+  // quarter-warp reads fall on disjoint bank halves.  Lane t copies chunk
+  // t % 8 of its rows with 16-byte cp.async; one commit group per leaf.
+  const bool a_staged = p.a_staged != 0;
+  const int slot_rows = a_staged ? 16 : 16 + NGW;
+  const int slot_bytes = slot_rows * 128;
+  uint8_t *sa = reinterpret_cast<uint8_t *>(smem_f4) + p.a_offset;      // [r][lc * 128]
+  uint8_t *ring = reinterpret_cast<uint8_t *>(smem_f4) + p.ring_offset + (size_t)warp * PF * slot_bytes;
+  const int a_stride = p.lc * 128;
+  if (a_staged) {
+    // A rows [adapter][j][split*lc*64 ...) -> sa[j][...], all threads
+    const int pieces = p.r * p.lc * 8;
+    const uint16_t *a0 = p.at + (size_t)ti.adapter * p.r * p.K + (size_t)split * p.lc * kLeaf;
+    for (int pc = threadIdx.x; pc < pieces; pc += blockDim.x) {
+      const int j = pc / (p.lc * 8), ch = pc % (p.lc * 8);    // row, 16-byte chunk in the row
+      const int sw = (ch & ~7) | ((ch & 7) ^ ((j & 1) << 2));
+      cp_async16(sa + (size_t)j * a_stride + sw * 16, a0 + (size_t)j * p.K + ch * 8);
+    }
+  }
+  cp_async_commit();                                 // group: A slice (possibly empty)
+
+  constexpr int MAXP = (16 + NGW) * 8 / 32;          // pieces per lane per leaf (upper bound)
+  const int npieces = slot_rows * 8 / 32;
+  const int pc = lane & 7;                           // chunk this lane copies
+  const uint16_t *src_row[MAXP];
+  uint32_t dst_off[MAXP];
+  bool src_ok[MAXP];
 #pragma unroll
-  for (int t = 0; t < NT; t++)
-    acol[t] = p.at + ((size_t)ti.adapter * p.r + ng * NGW + t * 8 + g) * p.K + 8 * c;
+  for (int u = 0; u < MAXP; u++) {
+    const int q = (lane >> 3) + 4 * u;               // slot row
+    dst_off[u] = (uint32_t)(q * 128 + ((pc ^ ((q & 1) << 2)) << 4));
+    src_ok[u] = u < npieces;
+    src_row[u] = p.x;
+    if (q < 16) {
+      const int lr = mt * 16 + q;
+      src_ok[u] = lr < ti.rows;
+      const int row = src_ok[u] ? (p.perm ? p.perm[ti.seg_begin + ti.row0 + lr] : ti.row0 + lr) : 0;
+      src_row[u] = p.x + (size_t)row * p.K + 8 * pc;
+    } else if (src_ok[u]) {
+      src_row[u] = p.at + ((size_t)ti.adapter * p.r + ng * NGW + (q - 16)) * p.K + 8 * pc;
+    }
+  }
+  auto issue_leaf = [&](int slot, int leaf) {
+    uint8_t *base = ring + (size_t)slot * slot_bytes;
+#pragma unroll
+    for (int u = 0; u < MAXP; u++)
+      if (src_ok[u]) cp_async16(base + dst_off[u], src_row[u] + (size_t)leaf * kLeaf);
+  };
+  const int swz = (g & 1) << 2;
 
   // ---- this warp's leaves: [leaf0, leaf0 + lg), folded in post order
   const int leaf0 = split * p.lc + lgi * p.lg;
@@ -162,12 +197,37 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
       for (int q = 0; q < 4; q++) st[d][t][q] = 0.0f;
   int depth = 0;
 
-  LeafFrag<NT> cur, nxt;
-  load_leaf<NT>(cur, xr0, xr1, v0, v1, acol, leaf0 * kLeaf);
+#pragma unroll
+  for (int j = 0; j < PF; j++) {
+    if (j < p.lg) issue_leaf(j, leaf0 + j);
+    cp_async_commit();
+  }
+  if (a_staged) {
+    cp_async_wait<PF>();                             // this thread's A pieces
+    __syncthreads();                                 // everyone's
+  }
   for (int i = 0; i < p.lg; i++) {
-    if (i + 1 < p.lg) load_leaf<NT>(nxt, xr0, xr1, v0, v1, acol, (leaf0 + i + 1) * kLeaf);
+    cp_async_wait<PF - 1>();                         // leaf i has landed (this lane's pieces)
+    __syncwarp();                                    // ... and every lane's
+    const uint8_t *slot = ring + (size_t)(i % PF) * slot_bytes;
+    const int li = lgi * p.lg + i;                   // leaf index inside the CTA's split
+    LeafFrag<NT> f;
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int ch = ((h * 4 + c) ^ swz) << 4;
+      f.xa[h][0] = v0 ? *reinterpret_cast<const uint4 *>(slot + g * 128 + ch) : make_uint4(0, 0, 0, 0);
+      f.xa[h][1] = v1 ? *reinterpret_cast<const uint4 *>(slot + (g + 8) * 128 + ch) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+        f.ab[h][t] = a_staged
+            ? *reinterpret_cast<const uint4 *>(sa + (size_t)(ng * NGW + t * 8 + g) * a_stride + li * 128 + ch)
+            : *reinterpret_cast<const uint4 *>(slot + (16 + t * 8 + g) * 128 + ch);
+    }
+    __syncwarp();                                    // slot consumed by every lane
+    if (i + PF < p.lg) issue_leaf(i % PF, leaf0 + i + PF);
+    cp_async_commit();
     float acc[NT][4];
-    mma_leaf<NT>(acc, cur);
+    mma_leaf<NT>(acc, f);
     // push (register stack: every index is a compile-time constant, the
     // slot is chosen by predication)
 #pragma unroll
@@ -196,8 +256,8 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
       }
       depth--;
     }
-    cur = nxt;
   }
+  cp_async_wait<0>();
   if (depth != 1) flag_error(p.status, BI_ERR_INVALID_ARG);   // schedule inconsistent
 
   // ---- group values -> shared memory, element (local row, column)
@@ -288,10 +348,10 @@ static int tree_merge_schedule(int n, uint8_t *merges) {
   return maxd;
 }
 
-template <int NGW, int MAXD>
+template <int NGW, int MAXD, int PF>
 static cudaError_t launch_shrink_t(const ShrinkParams &p, int tiles, int threads, size_t smem,
                                    cudaStream_t stream) {
-  auto kern = shrink_kernel<NGW, MAXD>;
+  auto kern = shrink_kernel<NGW, MAXD, PF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -347,14 +407,15 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
 
   const int ngw = (r % 16 == 0) ? 16 : 8;
   p.ngroups = r / ngw;
-  // m-tiles per CTA: up to 4 (64 rows), fewer when the batch is small
-  int mt = std::min(4, (M + 15) / 16);
-  while (mt > 1 && mt * p.ngroups > 8) mt >>= 1;
+  // Tiling (bit-neutral).  Leaf groups first: enough warps per row tile
+  // that each walks at most 8 leaves (a power of two dividing the split's
+  // leaves); then up to 4 row tiles of 16, at most 8 warps per CTA.
   if (p.ngroups > 8) return BI_ERR_UNSUPPORTED_SHAPE;
-  p.mtiles = mt;
-  // leaf groups: fill up to 8 warps, power of two dividing lc
   int G = 1;
-  while (G * 2 * mt * p.ngroups <= 8 && p.lc % (G * 2) == 0) G *= 2;
+  while (p.lc / G > 8 && p.lc % (G * 2) == 0 && G * 2 * p.ngroups <= 8) G *= 2;
+  int mt = std::min(4, (M + 15) / 16);
+  while (mt > 1 && mt * G * p.ngroups > 8) mt >>= 1;
+  p.mtiles = mt;
   p.groups = G;
   p.lg = p.lc / G;
   if (p.lg > kMaxGroupLeaves) return BI_ERR_UNSUPPORTED_SHAPE;
@@ -362,22 +423,33 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   const int warps = G * mt * p.ngroups;
   const int threads = 32 * warps;
   const int bm = 16 * mt;
-  const size_t smem = (size_t)G * bm * r * sizeof(float);
+  const int pf = p.lg >= 2 ? 2 : 1;
+  const size_t part_bytes = ((size_t)G * bm * r * sizeof(float) + 127) & ~size_t(127);
+  const size_t a_bytes = (size_t)r * p.lc * 128;
+  p.a_staged = a_bytes <= 64 * 1024 ? 1 : 0;
+  p.a_offset = (int)part_bytes;
+  const int slot_bytes = (p.a_staged ? 16 : 16 + ngw) * 128;
+  p.ring_offset = (int)(part_bytes + (p.a_staged ? ((a_bytes + 127) & ~size_t(127)) : 0));
+  const size_t smem = (size_t)p.ring_offset + (size_t)warps * pf * slot_bytes;
   const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
 
   if (mode == BI_SHRINK_ATOMIC) {
     BI_CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)M * r * sizeof(float), stream));
   }
   cudaError_t e;
+#define BI_SHRINK_PF(NGW_, MAXD_)                                                   \
+  (pf == 2 ? launch_shrink_t<NGW_, MAXD_, 2>(p, tiles, threads, smem, stream)       \
+            : launch_shrink_t<NGW_, MAXD_, 1>(p, tiles, threads, smem, stream))
   if (ngw == 16) {
-    if (depth <= 4) e = launch_shrink_t<16, 4>(p, tiles, threads, smem, stream);
-    else if (depth <= 8) e = launch_shrink_t<16, 8>(p, tiles, threads, smem, stream);
-    else e = launch_shrink_t<16, 12>(p, tiles, threads, smem, stream);
+    if (depth <= 4) e = BI_SHRINK_PF(16, 4);
+    else if (depth <= 8) e = BI_SHRINK_PF(16, 8);
+    else e = BI_SHRINK_PF(16, 12);
   } else {
-    if (depth <= 4) e = launch_shrink_t<8, 4>(p, tiles, threads, smem, stream);
-    else if (depth <= 8) e = launch_shrink_t<8, 8>(p, tiles, threads, smem, stream);
-    else e = launch_shrink_t<8, 12>(p, tiles, threads, smem, stream);
+    if (depth <= 4) e = BI_SHRINK_PF(8, 4);
+    else if (depth <= 8) e = BI_SHRINK_PF(8, 8);
+    else e = BI_SHRINK_PF(8, 12);
   }
+#undef BI_SHRINK_PF
   return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -395,7 +395,7 @@ void or_log_softmax_exact(const float *x, long R, long n, double *out, int nthre
 }
 
 /* Canonical fp32, two passes: m = row max (exact in any order);
- * d_k = x_k - m; S = canon_sum(or_exp(d_k); T=1024, V=4); L = or_log(S);
+ * d_k = x_k - m; S = canon_sum(or_exp(d_k); T=4096, V=4); L = or_log(S);
  * out_k = d_k - L. */
 void or_log_softmax_canon(const float *x, long R, long n, float *out, int nthreads)
 {
@@ -406,7 +406,7 @@ void or_log_softmax_canon(const float *x, long R, long n, float *out, int nthrea
         for (long k = 1; k < n; k++) if (xr[k] > m) m = xr[k];
         float *e = (float *)malloc(sizeof(float) * (size_t)n);
         for (long k = 0; k < n; k++) e[k] = or_exp(xr[k] - m);
-        float S = or_canon_sum(e, n, 1024, 4);
+        float S = or_canon_sum(e, n, 4096, 4);
         float L = or_log(S);
         for (long k = 0; k < n; k++) out[i * n + k] = (xr[k] - m) - L;
         free(e);

@@ -351,7 +351,7 @@ def test_log_softmax_canon_closed_forms(oracle_mod):
 
 
 def test_log_softmax_canon_sum_order(oracle_mod):
-    """n = 8192, T = 1024 lanes of V = 4.  x[0] = 0 is the max (term 1),
+    """n = 8192, T = 4096 lanes of V = 4.  x[0] = 0 is the max (term 1),
     x[4..7] = -17 (term eps = exp(-17) ~ 4.1e-8, below half an ulp of 1),
     every other logit -200 (term 0).  Lane 0 holds elements 0..3: 1.
     Lane 1 holds elements 4..7: c = ((eps + eps) + eps) + eps ~ 1.7e-7.
@@ -371,6 +371,25 @@ def test_log_softmax_canon_sum_order(oracle_mod):
     assert f32bits(out[0]) == f32bits(F32(F32(0.0) - L))
     assert f32bits(out[5]) == f32bits(F32(F32(-17.0) - L))
     assert f32bits(out[9]) == f32bits(F32(F32(-200.0) - L))
+
+
+def test_log_softmax_canon_lane_count(oracle_mod):
+    """Pins T = 4096: n = 8192, x[0] = 0 (term 1), x[4096..4099] = -17
+    (vector 1024, terms eps), rest -200 (terms 0).  With 4096 lanes vector
+    1024 is lane 1024, its own chain: c = four eps, S = fl(1 + c) = 1 + 2^-23,
+    L != 0 and out[0] = -L.  With 1024 lanes it would be lane 0 again and be
+    absorbed into 1 (L = 0, out[0] = 0)."""
+    n = 8192
+    x = np.full((1, n), -200.0, np.float32)
+    x[0, 0] = 0.0
+    x[0, 4096:4100] = -17.0
+    eps = oracle_mod.exp_spec(-17.0)
+    c = F32(F32(F32(F32(F32(0) + eps) + eps) + eps) + eps)
+    L = oracle_mod.log_spec(F32(F32(1.0) + c))
+    assert L != 0
+    out = oracle_mod.log_softmax_canon(x)[0]
+    assert f32bits(out[0]) == f32bits(F32(F32(0.0) - L))
+    assert f32bits(out[4097]) == f32bits(F32(F32(-17.0) - L))
 
 
 def test_log_softmax_canon_vs_exact(oracle_mod):

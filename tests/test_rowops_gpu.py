@@ -88,6 +88,25 @@ def test_log_softmax_shapes(n):
     assert np.array_equal(lsm(x), oracle.log_softmax_canon(x).view(np.uint32))
 
 
+def test_log_softmax_wide_range_rows():
+    """Logits spread over hundreds: many vectors take the general exp path
+    (x - max < -87, down to the flush to zero below -103)."""
+    x = synth.normal_f32((7, 151936), 60.0, seed=77)
+    x[3, ::5] = -1e4
+    assert np.array_equal(lsm(x), oracle.log_softmax_canon(x).view(np.uint32))
+
+
+def test_exp_shortcut_matches_exp():
+    """The log_softmax exp shortcut gives bi_exp's bits on [-87, 88]."""
+    xs = np.concatenate([np.linspace(-87, 88, 1 << 20), -np.abs(np.random.default_rng(4).standard_normal(1 << 18) * 30)])
+    xs = xs[(xs >= -87) & (xs <= 88)].astype(np.float32)
+    a = torch.empty(xs.size, dtype=torch.float32, device="cuda")
+    b = torch.empty_like(a)
+    bi.math_spec(dev(xs), a, "exp")
+    bi.math_spec(dev(xs), b, "exp_fast")
+    assert np.array_equal(host_bits(a), host_bits(b))
+
+
 def test_log_softmax_closed_form():
     x = np.full((2, 151936), 1.5, np.float32)
     out = lsm(x).view(np.float32)
