@@ -198,8 +198,7 @@ __global__ void __launch_bounds__(1024)
 log_softmax_kernel(const __grid_constant__ LsmParams p) {
   extern __shared__ float4 lsm_smem[];
   __shared__ float s_red[32];
-  __shared__ float s_max, s_sum;
-  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ float s_max, s_sum, s_bcast, s_bcast2;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C;
   const int q = (int)cluster.block_rank();
@@ -215,16 +214,11 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   const int nj = lane_id < nvec ? (nvec - 1 - lane_id) / kLsmT + 1 : 0;
 
   // ---- this lane's vectors -> its shared-memory slots: 16-byte cp.async
-  // copies, all in flight at once; each thread's arrival on the barrier
-  // fires when its copies have landed.
-  if (tau == 0) {
-    mbar_init(&s_bar, blockDim.x);
-    mbar_fence_init();
-  }
-  __syncthreads();
+  // copies, all in flight at once.  Each thread reads back only its own
+  // slots, so waiting for its own copies is enough.
   for (int j = 0; j < nj; j++) cp_async16(lsm_smem + (size_t)j * lpc + tau, xr + (size_t)j * kLsmT + lane_id);
-  cp_async_arrive(&s_bar);
-  if (!mbar_wait(&s_bar, 0)) flag_error(p.status, BI_ERR_TIMEOUT);
+  cp_async_commit();
+  cp_async_wait<0>();
 
   // ---- local max
   float m = -INFINITY;
@@ -240,10 +234,16 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     v = warp_max(v);
     if (tau == 0) s_max = v;
   }
-  cluster.sync();
-  // row max over the cluster (max is exact in any order)
-  float rmax = -INFINITY;
-  for (int r = 0; r < C; r++) rmax = fmaxf(rmax, *cluster.map_shared_rank(&s_max, r));
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  // row max over the cluster (exact in any order): warp 0 gathers, all read
+  if (tau < 32) {
+    float v = tau < C ? *cluster.map_shared_rank(&s_max, tau) : -INFINITY;
+    v = warp_max(v);
+    if (tau == 0) s_bcast = v;
+  }
+  __syncthreads();
+  const float rmax = s_bcast;
 
   // ---- lane chain of bi_exp(x - max); d = x - max stays in the slot
   float s = 0.0f;
@@ -262,7 +262,6 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     s = __fadd_rn(s, e.w);
   }
   s = warp_tree_sum(s);
-  __syncthreads();                      // s_red reuse
   if ((tau & 31) == 0) s_red[tau >> 5] = s;
   __syncthreads();
   if (tau < 32) {
@@ -270,17 +269,18 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     for (int o = 1; o < nwarps; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
     if (tau == 0) s_sum = v;
   }
-  cluster.sync();
-  // perfect tree over the C CTA subtrees (every CTA computes the same bits)
-  float part[16];
-#pragma unroll
-  for (int r = 0; r < 16; r++) part[r] = r < C ? *cluster.map_shared_rank(&s_sum, r) : 0.0f;
-#pragma unroll
-  for (int st = 1; st < 16; st <<= 1)
-#pragma unroll
-    for (int r = 0; r + st < 16; r += 2 * st)
-      if (r + st < C) part[r] = __fadd_rn(part[r], part[r + st]);
-  const float L = bi_log(part[0]);
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  // perfect tree over the C CTA subtrees: warp 0 gathers them into lanes
+  // 0..C-1 and adds with the xor butterfly (pairs, then pairs of pairs)
+  if (tau < 32) {
+    float v = tau < C ? *cluster.map_shared_rank(&s_sum, tau) : 0.0f;
+    for (int o = 1; o < C; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (tau == 0) s_bcast2 = bi_log(v);
+  }
+  __syncthreads();
+  cluster_arrive_relaxed();               // done reading the peers' shared memory
+  const float L = s_bcast2;
 
   // ---- write out = d - L
   for (int j = 0; j < nj; j++) {
@@ -292,7 +292,7 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     o.w = __fsub_rn(d.w, L);
     __stcs(outr + (size_t)j * kLsmT + lane_id, o);
   }
-  cluster.sync();   // peers may still read s_max / s_sum of this CTA
+  cluster_wait();                         // keep s_max / s_sum alive until the peers are done
 }
 
 // Test and reference hook: the library's exp / log applied elementwise.

@@ -61,7 +61,6 @@ struct ShrinkParams {
   int mode;
   int a_staged;             // 1: the CTA's A slice sits in shared memory
   int a_offset;             // bytes from the start of dynamic shared memory to the A slice
-  int ring_offset;          // bytes from the start of dynamic shared memory to the warp rings
   uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
 };
 
@@ -96,7 +95,7 @@ BI_DEV void mma_leaf(float acc[NT][4], const LeafFrag<NT> &f) {
   }
 }
 
-template <int NGW, int MAXD, int PF>
+template <int NGW, int MAXD, int PF, bool ASTAGED>
 __global__ void __launch_bounds__(256)
 shrink_kernel(const __grid_constant__ ShrinkParams p) {
   constexpr int NT = NGW / 8;
@@ -134,16 +133,12 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   const int lr0 = mt * 16 + g, lr1 = lr0 + 8;       // local rows in the tile
   const bool v0 = lr0 < ti.rows, v1 = lr1 < ti.rows;
 
-  // ---- shared memory: the CTA's A slice (staged once when it fits) and a
-  // per-warp ring of PF leaf slots.  Rows are 128 bytes per leaf; the
-  // 16-byte chunk index is XOR-ed with (row & 1) << 2 so that the two rows a
-  // quarter-warp reads fall on disjoint bank halves.  Lane t copies chunk
-  // t % 8 of its rows with 16-byte cp.async; one commit group per leaf.
-  const bool a_staged = p.a_staged != 0;
-  const int slot_rows = a_staged ? 16 : 16 + NGW;
-  const int slot_bytes = slot_rows * 128;
+  // ---- shared memory holds the CTA's A slice (staged once, by every
+  // thread with 16-byte cp.async, when it fits in 64 KB).  Rows are 128 bytes
+  // per leaf; the 16-byte chunk index is XOR-ed with (row & 1) << 2 so that
+  // the two rows a quarter-warp reads fall on disjoint bank halves.
+  constexpr bool a_staged = ASTAGED;
   uint8_t *sa = reinterpret_cast<uint8_t *>(smem_f4) + p.a_offset;      // [r][lc * 128]
-  uint8_t *ring = reinterpret_cast<uint8_t *>(smem_f4) + p.ring_offset + (size_t)warp * PF * slot_bytes;
   const int a_stride = p.lc * 128;
   if (a_staged) {
     // A rows [adapter][j][split*lc*64 ...) -> sa[j][...], all threads
@@ -155,34 +150,31 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
       cp_async16(sa + (size_t)j * a_stride + sw * 16, a0 + (size_t)j * p.K + ch * 8);
     }
   }
-  cp_async_commit();                                 // group: A slice (possibly empty)
+  cp_async_commit();
 
-  constexpr int MAXP = (16 + NGW) * 8 / 32;          // pieces per lane per leaf (upper bound)
-  const int npieces = slot_rows * 8 / 32;
-  const int pc = lane & 7;                           // chunk this lane copies
-  const uint16_t *src_row[MAXP];
-  uint32_t dst_off[MAXP];
-  bool src_ok[MAXP];
+  // x fragment rows g and g+8 of this warp's m-tile, read straight from
+  // global memory into a register ring of PF leaves; A fragments come from
+  // the staged slice, or from global memory with the x ones when A is not
+  // staged.
+  int row0 = 0, row1 = 0;
+  if (v0) row0 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr0] : ti.row0 + lr0;
+  if (v1) row1 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr1] : ti.row0 + lr1;
+  const uint16_t *xr0 = p.x + (size_t)row0 * p.K + 8 * c;
+  const uint16_t *xr1 = p.x + (size_t)row1 * p.K + 8 * c;
+  const uint16_t *acol[NT];
 #pragma unroll
-  for (int u = 0; u < MAXP; u++) {
-    const int q = (lane >> 3) + 4 * u;               // slot row
-    dst_off[u] = (uint32_t)(q * 128 + ((pc ^ ((q & 1) << 2)) << 4));
-    src_ok[u] = u < npieces;
-    src_row[u] = p.x;
-    if (q < 16) {
-      const int lr = mt * 16 + q;
-      src_ok[u] = lr < ti.rows;
-      const int row = src_ok[u] ? (p.perm ? p.perm[ti.seg_begin + ti.row0 + lr] : ti.row0 + lr) : 0;
-      src_row[u] = p.x + (size_t)row * p.K + 8 * pc;
-    } else if (src_ok[u]) {
-      src_row[u] = p.at + ((size_t)ti.adapter * p.r + ng * NGW + (q - 16)) * p.K + 8 * pc;
+  for (int t = 0; t < NT; t++)
+    acol[t] = p.at + ((size_t)ti.adapter * p.r + ng * NGW + t * 8 + g) * p.K + 8 * c;
+  auto load_leaf = [&](LeafFrag<NT> &f, int leaf) {
+    const size_t k = (size_t)leaf * kLeaf;
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      f.xa[h][0] = v0 ? ldg128_stream(xr0 + k + 32 * h) : make_uint4(0, 0, 0, 0);
+      f.xa[h][1] = v1 ? ldg128_stream(xr1 + k + 32 * h) : make_uint4(0, 0, 0, 0);
+      if (!a_staged)
+#pragma unroll
+        for (int t = 0; t < NT; t++) f.ab[h][t] = ldg128(acol[t] + k + 32 * h);
     }
-  }
-  auto issue_leaf = [&](int slot, int leaf) {
-    uint8_t *base = ring + (size_t)slot * slot_bytes;
-#pragma unroll
-    for (int u = 0; u < MAXP; u++)
-      if (src_ok[u]) cp_async16(base + dst_off[u], src_row[u] + (size_t)leaf * kLeaf);
   };
   const int swz = (g & 1) << 2;
 
@@ -197,67 +189,64 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
       for (int q = 0; q < 4; q++) st[d][t][q] = 0.0f;
   int depth = 0;
 
+  LeafFrag<NT> ring[PF];
 #pragma unroll
-  for (int j = 0; j < PF; j++) {
-    if (j < p.lg) issue_leaf(j, leaf0 + j);
-    cp_async_commit();
-  }
+  for (int j = 0; j < PF; j++)
+    if (j < p.lg) load_leaf(ring[j], leaf0 + j);
   if (a_staged) {
-    cp_async_wait<PF>();                             // this thread's A pieces
+    cp_async_wait<0>();                              // this thread's A pieces
     __syncthreads();                                 // everyone's
   }
-  for (int i = 0; i < p.lg; i++) {
-    cp_async_wait<PF - 1>();                         // leaf i has landed (this lane's pieces)
-    __syncwarp();                                    // ... and every lane's
-    const uint8_t *slot = ring + (size_t)(i % PF) * slot_bytes;
-    const int li = lgi * p.lg + i;                   // leaf index inside the CTA's split
-    LeafFrag<NT> f;
+  for (int i0 = 0; i0 < p.lg; i0 += PF) {
 #pragma unroll
-    for (int h = 0; h < 2; h++) {
-      const int ch = ((h * 4 + c) ^ swz) << 4;
-      f.xa[h][0] = v0 ? *reinterpret_cast<const uint4 *>(slot + g * 128 + ch) : make_uint4(0, 0, 0, 0);
-      f.xa[h][1] = v1 ? *reinterpret_cast<const uint4 *>(slot + (g + 8) * 128 + ch) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < PF; j++) {
+      const int i = i0 + j;
+      if (i < p.lg) {
+        LeafFrag<NT> f = ring[j];
+        if (a_staged) {
+          const int li = lgi * p.lg + i;             // leaf index inside the CTA's split
 #pragma unroll
-      for (int t = 0; t < NT; t++)
-        f.ab[h][t] = a_staged
-            ? *reinterpret_cast<const uint4 *>(sa + (size_t)(ng * NGW + t * 8 + g) * a_stride + li * 128 + ch)
-            : *reinterpret_cast<const uint4 *>(slot + (16 + t * 8 + g) * 128 + ch);
-    }
-    __syncwarp();                                    // slot consumed by every lane
-    if (i + PF < p.lg) issue_leaf(i % PF, leaf0 + i + PF);
-    cp_async_commit();
-    float acc[NT][4];
-    mma_leaf<NT>(acc, f);
-    // push (register stack: every index is a compile-time constant, the
-    // slot is chosen by predication)
+          for (int h = 0; h < 2; h++) {
+            const int ch = ((h * 4 + c) ^ swz) << 4;
 #pragma unroll
-    for (int d = 0; d < MAXD; d++) {
-      const bool hit = d == depth;
-#pragma unroll
-      for (int t = 0; t < NT; t++)
-#pragma unroll
-        for (int q = 0; q < 4; q++) st[d][t][q] = hit ? acc[t][q] : st[d][t][q];
-    }
-    depth++;
-    // merge the subtrees that end at this leaf: left = st[depth-2]
-    const int nm = p.merges[i];
-#pragma unroll 1
-    for (int m = 0; m < nm; m++) {
-#pragma unroll
-      for (int d = 1; d < MAXD; d++) {
-        const bool hit = d == depth - 1;
-#pragma unroll
-        for (int t = 0; t < NT; t++)
-#pragma unroll
-          for (int q = 0; q < 4; q++) {
-            const float sum = __fadd_rn(st[d - 1][t][q], st[d][t][q]);
-            st[d - 1][t][q] = hit ? sum : st[d - 1][t][q];
+            for (int t = 0; t < NT; t++)
+              f.ab[h][t] = *reinterpret_cast<const uint4 *>(sa + (size_t)(ng * NGW + t * 8 + g) * a_stride + li * 128 + ch);
           }
+        }
+        if (i + PF < p.lg) load_leaf(ring[j], leaf0 + i + PF);
+        float acc[NT][4];
+        mma_leaf<NT>(acc, f);
+        // push (register stack: every index is a compile-time constant, the
+        // slot is chosen by predication)
+#pragma unroll
+        for (int d = 0; d < MAXD; d++) {
+          const bool hit = d == depth;
+#pragma unroll
+          for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) st[d][t][q] = hit ? acc[t][q] : st[d][t][q];
+        }
+        depth++;
+        // merge the subtrees that end at this leaf: left = st[depth-2]
+        const int nm = p.merges[i];
+#pragma unroll 1
+        for (int m = 0; m < nm; m++) {
+#pragma unroll
+          for (int d = 1; d < MAXD; d++) {
+            const bool hit = d == depth - 1;
+#pragma unroll
+            for (int t = 0; t < NT; t++)
+#pragma unroll
+              for (int q = 0; q < 4; q++) {
+                const float sum = __fadd_rn(st[d - 1][t][q], st[d][t][q]);
+                st[d - 1][t][q] = hit ? sum : st[d - 1][t][q];
+              }
+          }
+          depth--;
+        }
       }
-      depth--;
     }
   }
-  cp_async_wait<0>();
   if (depth != 1) flag_error(p.status, BI_ERR_INVALID_ARG);   // schedule inconsistent
 
   // ---- group values -> shared memory, element (local row, column)
@@ -351,7 +340,7 @@ static int tree_merge_schedule(int n, uint8_t *merges) {
 template <int NGW, int MAXD, int PF>
 static cudaError_t launch_shrink_t(const ShrinkParams &p, int tiles, int threads, size_t smem,
                                    cudaStream_t stream) {
-  auto kern = shrink_kernel<NGW, MAXD, PF>;
+  auto kern = p.a_staged ? shrink_kernel<NGW, MAXD, PF, true> : shrink_kernel<NGW, MAXD, PF, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -428,9 +417,7 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   const size_t a_bytes = (size_t)r * p.lc * 128;
   p.a_staged = a_bytes <= 64 * 1024 ? 1 : 0;
   p.a_offset = (int)part_bytes;
-  const int slot_bytes = (p.a_staged ? 16 : 16 + ngw) * 128;
-  p.ring_offset = (int)(part_bytes + (p.a_staged ? ((a_bytes + 127) & ~size_t(127)) : 0));
-  const size_t smem = (size_t)p.ring_offset + (size_t)warps * pf * slot_bytes;
+  const size_t smem = part_bytes + (p.a_staged ? a_bytes : 0);
   const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
 
   if (mode == BI_SHRINK_ATOMIC) {
