@@ -18,7 +18,7 @@ The headline `value` is the deterministic split-K LoRA-shrink HBM GB/s on
 the segmented workload (algorithmic bytes / kernel time, CUDA events on the
 launch stream).  Every kernel's own time, throughput and roofline fraction
 is listed under "kernels"; "roofline" describes the kernel with the largest
-share of the step.  L2 is flushed (a 256 MiB memset) before each kernel.
+share of the step.  L2 is flushed before each kernel: 256 MiB written, then read back.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -162,6 +162,8 @@ class Workload:
         self.lsm = torch.empty_like(self.logits)
         self.mean = torch.empty(4096, dtype=torch.float32, device="cuda")
         self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.flush_f = self.flush.view(torch.float32)
+        self.flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
         self.kernels = self._kernels()
 
     def _kernels(self):
@@ -238,9 +240,17 @@ def run_ours(args, rank, world, device):
     pk = peaks()
     cs = torch.cuda.Stream()                       # capture / launch stream
 
+    def flush_l2(i):
+        # 256 MiB written, then read back: the write evicts every line the
+        # last kernel left, the read-back makes the write-backs of that
+        # buffer happen here, so the next kernel starts on a cold L2 holding
+        # only clean lines and its DRAM traffic is its own
+        wl.flush.fill_(i & 0xff)
+        torch.sum(wl.flush_f, dim=0, out=wl.flush_sink)
+
     def step_body():
         for i, (name, fn, *_rest) in enumerate(wl.kernels):
-            wl.flush.fill_(i & 0xff)               # L2 flush: 256 MiB write
+            flush_l2(i)
             fn()
 
     # everything below runs with cs as the current stream: graph replays go to
@@ -261,7 +271,7 @@ def run_ours(args, rank, world, device):
         def reps(fn):
             def body():
                 for i in range(R):
-                    wl.flush.fill_(i & 0xff)
+                    flush_l2(i)
                     if fn is not None:
                         fn()
             return body
@@ -343,7 +353,7 @@ def run_ours(args, rank, world, device):
         "data": "synthetic (seeded numpy PCG64; shapes of the pages' workloads)",
         "config": {"workload": WORKLOAD, "global_batch": M4 * world, "seq_len": None,
                    "parallelism": f"dp{world} (independent replicas, no collective)",
-                   "l2": "flushed before every kernel (256 MiB write)",
+                   "l2": "flushed before every kernel (256 MiB written, then read back: cold, clean L2)",
                    "timing": "step = one CUDA-graph replay of the whole path; per-kernel time = "
                              f"(graph of {R} x [flush, kernel]) - (graph of {R} x [flush]), CUDA events"},
         "roofline": {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"],

@@ -227,7 +227,9 @@ bi_status bi_mean(const float *x, float *out, int rows, int n, bi_stream_t strea
  * applied elementwise: y[i] = bi_exp(x[i]) or bi_log(x[i]).  x, y fp32 [n].
  * bi_log is defined for positive normal x; bi_exp for x <= 88.  which = 2
  * runs the shortcut of bi_exp that log_softmax takes for -87 <= x <= 88
- * (same bits as bi_exp there; undefined outside). */
+ * (same bits as bi_exp there; undefined outside); which = 3 the same
+ * shortcut on packed two-lane fp32 instructions (elements 2k and 2k+1 form
+ * one pair).  Other values of which: BI_ERR_INVALID_ARG. */
 bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream);
 
 /* ------------------------------------------------------------------ */

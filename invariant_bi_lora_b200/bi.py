@@ -297,10 +297,11 @@ def mean(x, out, stream=None):
 
 def math_spec(x, y, which, stream=None):
     """y = the library's exp (which='exp'), log ('log') or the exp shortcut
-    log_softmax uses on [-87, 88] ('exp_fast') of x."""
+    log_softmax uses on [-87, 88] ('exp_fast'; 'exp_fast2' on packed two-lane
+    instructions) of x."""
     _check(x, "x", torch.float32)
     _check(y, "y", torch.float32)
-    _call("bi_math_spec", _ptr(x), _ptr(y), x.numel(), {"exp": 0, "log": 1, "exp_fast": 2}[which],
+    _call("bi_math_spec", _ptr(x), _ptr(y), x.numel(), {"exp": 0, "log": 1, "exp_fast": 2, "exp_fast2": 3}[which],
           _stream(stream))
     return y
 

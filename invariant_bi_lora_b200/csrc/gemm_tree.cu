@@ -7,17 +7,25 @@
 // same bits for every TP size.
 //
 // Order: K is cut into leaves of 256.  A leaf is one TMEM accumulation of
-// sixteen tcgen05.mma (M=128, N=64, K=16), restarted from zero for every
-// leaf.  Leaves are combined in fp32 by the canonical tree.  A shard (an
-// emulated TP rank) owns a contiguous block of L/shards leaves -- one
-// subtree -- and writes its partial; bi_tree_combine adds the top levels.
+// sixteen tcgen05.mma (M=128, K=16), restarted from zero for every leaf.
+// Leaves are combined in fp32 by the canonical tree.  A shard (an emulated
+// TP rank) owns a contiguous block of L/shards leaves -- one subtree -- and
+// writes its partial; bi_tree_combine adds the top levels.  The bits of an
+// accumulator element depend on its row of A, its row of W and the K order
+// only, not on the instruction's N, so the two tile widths below give the
+// same leaves (a test checks this against the batch-invariant GEMM).
 //
-// Per CTA (persistent, 320 threads): warp 0 issues TMA loads into an
-// 8-stage ring, warp 1 issues the MMAs into one of two 64-column TMEM leaf
-// buffers, warps 2..9 fold finished leaves into the pending stack of the
-// post-order tree walk.  The stack lives in TMEM too: 6 slots of 64 columns
-// (2 x 64 + 6 x 64 = 512 columns), enough for 64 leaves per shard.  Each
-// epilogue thread owns one row (its TMEM lane) and 32 of the 64 columns.
+// Per CTA (persistent, 320 threads): warp 0 issues TMA loads into a stage
+// ring, warp 1 issues the MMAs into one of two TMEM leaf buffers, warps
+// 2..9 fold finished leaves into the pending stack of the post-order tree
+// walk; each epilogue thread owns one row (its TMEM lane) and half of the
+// tile's columns.  Two layouts:
+//  * BN = 128, 1/2/4/8 leaves per shard (known at compile time): the walk is
+//    a binary counter; level 0 of the pending stack sits in registers,
+//    levels 1 and 2 in TMEM (2 x 128 buffer + 2 x 128 stack = 512 columns).
+//    The wide tile halves the operand bytes per flop that L2 must deliver.
+//  * BN = 64, any leaf count up to 64: the host-computed post-order schedule
+//    (merges per leaf), stack of 6 slots in TMEM (2 x 64 + 6 x 64 columns).
 #include "tc.cuh"
 
 #include <algorithm>
@@ -27,17 +35,22 @@ namespace bi {
 bi_status tree_combine_launch(const float *partials, float *out, int s, size_t count, cudaStream_t stream);
 
 namespace tg {
-constexpr int BM = 128, BN = 64, BK = 64, LEAF = 256, STAGES = 8;
+constexpr int BM = 128, BK = 64, LEAF = 256;
 constexpr int KB_PER_LEAF = LEAF / BK;                // 4
 constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                  // 8 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 24 KB
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);         // 320
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int STACK_SLOTS = 6;
+constexpr int STACK_SLOTS = 6;                        // BN = 64 layout
 constexpr int MAX_LEAVES = 64;                        // per shard
-constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int MAX_STAGES = 8;
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 64 ? 8 : 6;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+};
 }  // namespace tg
 
 struct TreeGemmParams {
@@ -48,18 +61,33 @@ struct TreeGemmParams {
 };
 
 struct TreeSmemTail {
-  uint64_t full[tg::STAGES];
-  uint64_t empty[tg::STAGES];
+  uint64_t full[tg::MAX_STAGES];
+  uint64_t empty[tg::MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint32_t tmem_base;
   uint32_t bail;
 };
 
+template <int N>
+BI_DEV void add_rn(float (&cur)[N], const float (&left)[N]) {
+#pragma unroll
+  for (int q = 0; q < N; q++) cur[q] = __fadd_rn(left[q], cur[q]);
+}
+
+// LPS = 0: BN = 64, any leaf count (p.merges).  LPS = 1, 2, 4, 8: BN = 128.
+template <int BN, int LPS>
 __global__ void __launch_bounds__(tg::THREADS, 1)
 gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ TreeGemmParams p) {
   using namespace tg;
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int B_BYTES = C::B_BYTES;
+  constexpr int STAGE_BYTES = C::STAGE_BYTES;
+  static_assert(LPS == 0 || BN == 128, "counter layout is the 128-wide tile");
+  static_assert(LPS != 0 || BN == 64, "schedule layout is the 64-wide tile");
+  constexpr int LOG2 = LPS >= 8 ? 3 : (LPS >= 4 ? 2 : (LPS >= 2 ? 1 : 0));
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sa = smem;
@@ -69,7 +97,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (p.M + BM - 1) / BM, tiles_n = p.N / BN;
   const int num_tiles = tiles_m * tiles_n * p.shards;
-  const int L = p.leaves;
+  const int L = LPS ? LPS : p.leaves;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
@@ -160,8 +188,8 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       }
     }
-  } else {
-    // ---------------- epilogue: post-order fold of the leaves
+  } else if constexpr (LPS == 0) {
+    // ---------------- epilogue: post-order fold of the leaves, stack in TMEM
     const int ew = warp - 2;
     const int quad = warp & 3;                  // TMEM lane quadrant of this warp
     const int half = ew >> 2;                   // which 32 of the 64 columns
@@ -175,7 +203,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       decode(tile, mb, nb, sh);
       int top = 0;
       for (int leaf = 0; leaf < L; leaf++) {
-        if (!mbar_wait(&tail->tfull[buf], buf_phase)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tail->tfull[buf], buf_phase))) {   // warp-uniform exit
           flag_error(p.status, BI_ERR_TIMEOUT);
           *bail = 1;
           break;
@@ -213,7 +241,97 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       }
     }
+  } else {
+    // ---------------- epilogue: binary counter over LPS leaves.  Leaf i
+    // closes the subtrees of the levels where its index has a 1 bit (left =
+    // the waiting subtree, right = the one just finished); at its lowest 0
+    // bit it parks the result.  Level 0 parks in registers, levels 1 and 2
+    // in TMEM columns 256 and 384.
+    const int ew = warp - 2;
+    const int quad = warp & 3;                  // TMEM lane quadrant of this warp
+    const int half = ew >> 2;                   // which 64 of the 128 columns
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    const uint32_t col_off = (uint32_t)(64 * half);
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (*bail) break;
+      int mb, nb, sh;
+      decode(tile, mb, nb, sh);
+      float lvl0[64];
+      float cur[64];
+      bool ok = true;
+#pragma unroll
+      for (int i = 0; i < LPS; i++) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tail->tfull[buf], buf_phase))) {   // warp-uniform exit
+          flag_error(p.status, BI_ERR_TIMEOUT);
+          *bail = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          uint32_t v0[32], v1[32];
+          const uint32_t src = tmem + lane_off + (uint32_t)(buf * BN) + col_off;
+          tmem_ld32(src, v0);
+          tmem_ld32(src + 32, v1);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tail->tempty[buf]);
+#pragma unroll
+          for (int q = 0; q < 32; q++) {
+            cur[q] = __uint_as_float(v0[q]);
+            cur[32 + q] = __uint_as_float(v1[q]);
+          }
+        }
+        if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+        if constexpr (LOG2 >= 1) {
+          if ((i & 1) == 0) {
+#pragma unroll
+            for (int q = 0; q < 64; q++) lvl0[q] = cur[q];
+            continue;
+          }
+          add_rn(cur, lvl0);
+#pragma unroll
+          for (int lv = 1; lv < LOG2; lv++) {
+            const uint32_t slot = tmem + lane_off + (uint32_t)(2 * BN + (lv - 1) * BN) + col_off;
+            if (((i >> lv) & 1) == 0) {
+              uint32_t w0[32], w1[32];
+#pragma unroll
+              for (int q = 0; q < 32; q++) {
+                w0[q] = __float_as_uint(cur[q]);
+                w1[q] = __float_as_uint(cur[32 + q]);
+              }
+              tmem_st32(slot, w0);
+              tmem_st32(slot + 32, w1);
+              break;
+            }
+            tmem_wait_st();                       // this thread's parked subtree has landed
+            uint32_t l0[32], l1[32];
+            tmem_ld32(slot, l0);
+            tmem_ld32(slot + 32, l1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; q++) {
+              cur[q] = __fadd_rn(__uint_as_float(l0[q]), cur[q]);
+              cur[32 + q] = __fadd_rn(__uint_as_float(l1[q]), cur[32 + q]);
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      const int row = mb * BM + 32 * quad + lane;
+      if (row < p.M) {
+        float *dst = p.out + ((size_t)sh * p.M + row) * p.N + nb * BN + 64 * half;
+#pragma unroll
+        for (int j = 0; j < 16; j++)
+          *reinterpret_cast<float4 *>(dst + 4 * j) = make_float4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
+      }
+    }
+    tmem_wait_st();
   }
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -238,7 +356,7 @@ static int schedule_depth(int n, const uint8_t *merges) {
 static bi_status tree_check(const void *A, const void *W, int M, int N, int K, int shards) {
   if (M < 0 || N <= 0 || K <= 0 || shards < 1) return BI_ERR_INVALID_ARG;
   if (M > 0 && (!A || !W)) return BI_ERR_INVALID_ARG;
-  if (K % tg::LEAF != 0 || N % tg::BN != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (K % tg::LEAF != 0 || N % 64 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
   const int L = K / tg::LEAF;
   if (!bi_pow2(shards) || L % shards != 0 || L / shards > tg::MAX_LEAVES) return BI_ERR_UNSUPPORTED_SHAPE;
   if (!bi_aligned16(A) || !bi_aligned16(W)) return BI_ERR_UNSUPPORTED_SHAPE;
@@ -255,18 +373,29 @@ static bi_status tree_partials_launch(const void *A, const void *W, float *out, 
   p.leaves = K / LEAF / shards;
   tree_schedule(p.leaves, p.merges);
   if (schedule_depth(p.leaves, p.merges) > STACK_SLOTS + 1) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int lps = p.leaves;
+  const bool wide = N % 128 == 0 && (lps == 1 || lps == 2 || lps == 4 || lps == 8);
+  const int bn = wide ? 128 : 64;
   CUtensorMap tmA, tmW;
   if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
-  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemm_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) != cudaSuccess)
-      return BI_ERR_CUDA;
-    attr_set = true;
-  }
-  const long tiles = (long)((M + BM - 1) / BM) * (N / BN) * shards;
+  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, bn)) return BI_ERR_CUDA;
+  const long tiles = (long)((M + BM - 1) / BM) * (N / bn) * shards;
   const int grid = (int)std::min<long>(tiles, num_sms());
-  gemm_tree_kernel<<<grid, THREADS, SMEM, stream>>>(tmA, tmW, p);
+  auto run = [&](auto kern, size_t smem) -> bool {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return false;
+    kern<<<grid, THREADS, smem, stream>>>(tmA, tmW, p);
+    return true;
+  };
+  bool ok;
+  switch (wide ? lps : 0) {
+    case 1: ok = run(gemm_tree_kernel<128, 1>, Cfg<128>::SMEM); break;
+    case 2: ok = run(gemm_tree_kernel<128, 2>, Cfg<128>::SMEM); break;
+    case 4: ok = run(gemm_tree_kernel<128, 4>, Cfg<128>::SMEM); break;
+    case 8: ok = run(gemm_tree_kernel<128, 8>, Cfg<128>::SMEM); break;
+    default: ok = run(gemm_tree_kernel<64, 0>, Cfg<64>::SMEM); break;
+  }
+  if (!ok) return BI_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

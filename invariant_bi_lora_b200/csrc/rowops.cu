@@ -178,13 +178,16 @@ struct LsmParams {
   int J;      // vector slots per lane = ceil(n/4 / 4096)
 };
 
+// bi_exp of the four lanes of d; the packed path when all four lie in
+// bi_exp_fast's range (d <= 0 here, so only the lower bound matters).
 BI_DEV float4 bi_exp4(float4 d) {
   float4 e;
-  if (fminf(fminf(d.x, d.y), fminf(d.z, d.w)) >= -87.0f) {
-    e.x = bi_exp_fast(d.x);
-    e.y = bi_exp_fast(d.y);
-    e.z = bi_exp_fast(d.z);
-    e.w = bi_exp_fast(d.w);
+  float mn;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(mn) : "f"(d.x), "f"(d.y), "f"(d.z));
+  if (fminf(mn, d.w) >= -87.0f) {
+    const float2 lo = upk2(bi_exp_fast2(pk2(d.x, d.y)));
+    const float2 hi = upk2(bi_exp_fast2(pk2(d.z, d.w)));
+    e = make_float4(lo.x, lo.y, hi.x, hi.y);
   } else {
     e.x = bi_exp(d.x);
     e.y = bi_exp(d.y);
@@ -192,6 +195,13 @@ BI_DEV float4 bi_exp4(float4 d) {
     e.w = bi_exp(d.w);
   }
   return e;
+}
+
+BI_DEV float max4(float m, float4 v) {
+  float a, b;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(a) : "f"(m), "f"(v.x), "f"(v.y));
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(b) : "f"(a), "f"(v.z), "f"(v.w));
+  return b;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -223,8 +233,7 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   // ---- local max
   float m = -INFINITY;
   for (int j = 0; j < nj; j++) {
-    const float4 v = lsm_smem[j * lpc + tau];
-    m = fmaxf(fmaxf(m, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+    m = max4(m, lsm_smem[j * lpc + tau]);
   }
   m = warp_max(m);
   if ((tau & 31) == 0) s_red[tau >> 5] = m;
@@ -243,17 +252,16 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     if (tau == 0) s_bcast = v;
   }
   __syncthreads();
-  const float rmax = s_bcast;
+  const uint64_t rmax2 = splat2(s_bcast);
 
   // ---- lane chain of bi_exp(x - max); d = x - max stays in the slot
   float s = 0.0f;
 #pragma unroll 2
   for (int j = 0; j < nj; j++) {
-    float4 d = lsm_smem[j * lpc + tau];
-    d.x = __fsub_rn(d.x, rmax);
-    d.y = __fsub_rn(d.y, rmax);
-    d.z = __fsub_rn(d.z, rmax);
-    d.w = __fsub_rn(d.w, rmax);
+    const float4 xv = lsm_smem[j * lpc + tau];
+    const float2 d01 = upk2(sub2_rn(pk2(xv.x, xv.y), rmax2));
+    const float2 d23 = upk2(sub2_rn(pk2(xv.z, xv.w), rmax2));
+    const float4 d = make_float4(d01.x, d01.y, d23.x, d23.y);
     lsm_smem[j * lpc + tau] = d;
     const float4 e = bi_exp4(d);
     s = __fadd_rn(s, e.x);
@@ -280,16 +288,14 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   }
   __syncthreads();
   cluster_arrive_relaxed();               // done reading the peers' shared memory
-  const float L = s_bcast2;
+  const uint64_t L2 = splat2(s_bcast2);
 
   // ---- write out = d - L
   for (int j = 0; j < nj; j++) {
     const float4 d = lsm_smem[j * lpc + tau];
-    float4 o;
-    o.x = __fsub_rn(d.x, L);
-    o.y = __fsub_rn(d.y, L);
-    o.z = __fsub_rn(d.z, L);
-    o.w = __fsub_rn(d.w, L);
+    const float2 o01 = upk2(sub2_rn(pk2(d.x, d.y), L2));
+    const float2 o23 = upk2(sub2_rn(pk2(d.z, d.w), L2));
+    const float4 o = make_float4(o01.x, o01.y, o23.x, o23.y);
     __stcs(outr + (size_t)j * kLsmT + lane_id, o);
   }
   cluster_wait();                         // keep s_max / s_sum alive until the peers are done
@@ -300,7 +306,13 @@ __global__ void math_spec_kernel(const float *__restrict__ x, float *__restrict_
                                  int which) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
-    y[i] = which == 0 ? bi_exp(x[i]) : (which == 1 ? bi_log(x[i]) : bi_exp_fast(x[i]));
+    if (which == 3) {                      // packed: elements 2k, 2k+1 share one pair
+      const size_t i0 = i & ~size_t(1), i1 = i0 + 1 < n ? i0 + 1 : i0;
+      const float2 e = upk2(bi_exp_fast2(pk2(x[i0], x[i1])));
+      y[i] = (i & 1) ? e.y : e.x;
+    } else {
+      y[i] = which == 0 ? bi_exp(x[i]) : (which == 1 ? bi_log(x[i]) : bi_exp_fast(x[i]));
+    }
 }
 
 }  // namespace bi
@@ -377,7 +389,7 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
 }
 
 extern "C" bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream) {
-  if ((n > 0 && (!x || !y)) || which < 0 || which > 2) return BI_ERR_INVALID_ARG;
+  if ((n > 0 && (!x || !y)) || which < 0 || which > 3) return BI_ERR_INVALID_ARG;
   if (n == 0) return BI_OK;
   const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16);
   bi::math_spec_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, which);

@@ -69,7 +69,7 @@ def test_other_rejects(libbi):
     assert libbi.bi_mean(FAKE, FAKE, -1, 8, None) == 1
     assert libbi.bi_tree_combine(FAKE, FAKE, 0, 16, None) == 1
     assert libbi.bi_tree_combine(FAKE, FAKE, 65, 16, None) == 1
-    assert libbi.bi_math_spec(FAKE, FAKE, 16, 3, None) == 1
+    assert libbi.bi_math_spec(FAKE, FAKE, 16, 4, None) == 1
     assert libbi.bi_selftest_bounded_wait(0, None) == 1
 
 

@@ -105,6 +105,11 @@ def test_exp_shortcut_matches_exp():
     bi.math_spec(dev(xs), a, "exp")
     bi.math_spec(dev(xs), b, "exp_fast")
     assert np.array_equal(host_bits(a), host_bits(b))
+    c = torch.empty_like(a)
+    bi.math_spec(dev(xs), c, "exp_fast2")              # packed pairs, both lanes
+    assert np.array_equal(host_bits(a), host_bits(c))
+    bi.math_spec(dev(xs[1:]), c[:-1], "exp_fast2")     # the other pairing
+    assert np.array_equal(host_bits(a)[1:], host_bits(c[:-1]))
 
 
 def test_log_softmax_closed_form():

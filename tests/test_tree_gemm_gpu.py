@@ -69,3 +69,16 @@ def test_tree_gemm_rejects():
     with pytest.raises(bi.BiError):
         bi.gemm_tree(a, w, C, shards=3)
     assert bi.get_device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,seed", [(300, 512, 1), (2048, 1024, 2)])
+def test_leaf_bits_independent_of_mma_width(M, N, seed):
+    """One 256-wide leaf: the batch-invariant GEMM (N=256 instructions) and
+    the tree GEMM (N=64 instructions) accumulate the same K order per output
+    element, so their bits agree; the tree GEMM's leaves rely on it."""
+    a, w = synth.gemm_inputs(M, N, 256, seed=seed)
+    A, W = dev_bf16(a), dev_bf16(w)
+    C1 = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    bi.gemm(A, W, C1)
+    C2 = tree(A, W, 1)
+    assert np.array_equal(host_bits(C1), host_bits(C2))
