@@ -125,6 +125,21 @@ BI_DEV TileInfo resolve_tile(const int32_t *offsets, int n_ad, int M, int tile, 
   return ti;
 }
 
+// resolve_tile for a whole CTA (every thread calls it): the n_ad + 2
+// segment starts are fetched by parallel loads into shared memory `s_off`
+// (room for kMaxAdapters + 2) and scanned there, so finding the tile costs
+// one memory round trip whatever its segment.  The result lands in *out
+// (shared) and is visible to every thread on return.
+constexpr int kMaxAdapters = 256;
+BI_DEV void resolve_tile_block(const int32_t *offsets, int n_ad, int M, int tile, int bm, int32_t *s_off,
+                               TileInfo *out) {
+  if (offsets)
+    for (int t = threadIdx.x; t < n_ad + 2; t += blockDim.x) s_off[t] = offsets[t];
+  __syncthreads();
+  if (threadIdx.x == 0) *out = resolve_tile(offsets ? s_off : nullptr, n_ad, M, tile, bm);
+  __syncthreads();
+}
+
 // Token index of position `pos` of a tile (identity without a plan).
 BI_DEV int tile_row(const int32_t *perm, const TileInfo &ti, int local) {
   return perm ? perm[ti.seg_begin + ti.row0 + local] : ti.row0 + local;

@@ -31,8 +31,8 @@ template <int KS>
 __global__ void __launch_bounds__(kExpThreads)
 expand_kernel(const __grid_constant__ ExpandParams p) {
   __shared__ TileInfo s_tile;
-  if (threadIdx.x == 0) s_tile = resolve_tile(p.offsets, p.n_ad, p.M, blockIdx.y, kExpBM);
-  __syncthreads();
+  __shared__ int32_t s_off[kMaxAdapters + 2];
+  resolve_tile_block(p.offsets, p.n_ad, p.M, blockIdx.y, kExpBM, s_off, &s_tile);
   const TileInfo ti = s_tile;
   if (ti.adapter < 0) return;
 

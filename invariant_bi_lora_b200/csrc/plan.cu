@@ -10,7 +10,6 @@
 namespace bi {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kMaxAdapters = 256;
 
 // One CTA.  Classes 0..n_ad-1 are adapters, class n_ad collects tokens whose
 // id is outside [0, n_ad).  Shared memory: counts / running bases

@@ -102,14 +102,14 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   extern __shared__ float4 smem_f4[];
   float *part = reinterpret_cast<float *>(smem_f4);     // [G][BM][r]
   __shared__ TileInfo s_tile;
+  __shared__ int32_t s_off[kMaxAdapters + 2];
 
   const int bm = 16 * p.mtiles;
   const int split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
 
-  if (threadIdx.x == 0) s_tile = resolve_tile(p.offsets, p.n_ad, p.M, blockIdx.y, bm);
-  __syncthreads();
+  resolve_tile_block(p.offsets, p.n_ad, p.M, blockIdx.y, bm, s_off, &s_tile);
   const TileInfo ti = s_tile;
   if (ti.adapter < 0) return;                       // uniform across the cluster
 
