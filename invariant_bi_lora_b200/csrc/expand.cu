@@ -28,7 +28,7 @@ struct ExpandParams {
 
 // KS = number of k16 steps (r rounded up to 16, / 16).
 template <int KS>
-__global__ void __launch_bounds__(kExpThreads)
+__global__ void __launch_bounds__(kExpThreads, 3)
 expand_kernel(const __grid_constant__ ExpandParams p) {
   __shared__ TileInfo s_tile;
   __shared__ int32_t s_off[kMaxAdapters + 2];
@@ -75,8 +75,13 @@ expand_kernel(const __grid_constant__ ExpandParams p) {
   }
 
   const uint16_t *bad = p.bt + (size_t)ti.adapter * p.N * p.r;
+  // The warp's 16 x 64 result goes through shared memory (row stride 72
+  // floats: the fragment writes are conflict-free per half-warp) and leaves
+  // as whole 256-byte row segments, two rows per store instruction.
+  __shared__ __align__(16) float s_out[kExpThreads / 32][16][72];
+  float (*so)[72] = s_out[warp];
   // B fragments of NB n-tiles at a time first (independent L2 loads in
-  // flight together), then their MMAs and stores
+  // flight together), then their MMAs
   constexpr int NB = KS <= 2 ? 8 : (KS <= 4 ? 4 : 2);
 #pragma unroll 1
   for (int nb0 = 0; nb0 < 8; nb0 += NB) {
@@ -95,31 +100,34 @@ expand_kernel(const __grid_constant__ ExpandParams p) {
     }
 #pragma unroll
     for (int i = 0; i < NB; i++) {
-      const int n0 = nbase + (nb0 + i) * 8;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int s = 0; s < KS; s++) mma_bf16_16816(acc, afr[s], bfr[i][s], acc);
-      const int n = n0 + 2 * c;
-      if (v0 && n0 < p.N) {
-        float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row0 * p.N + n);
-        float2 v = make_float2(acc[0], acc[1]);
-        if (p.accumulate) {
-          const float2 q = *o;
-          v.x = __fadd_rn(q.x, v.x);
-          v.y = __fadd_rn(q.y, v.y);
-        }
-        __stcs(o, v);
+      const int col = (nb0 + i) * 8 + 2 * c;
+      *reinterpret_cast<float2 *>(&so[g][col]) = make_float2(acc[0], acc[1]);
+      *reinterpret_cast<float2 *>(&so[g + 8][col]) = make_float2(acc[2], acc[3]);
+    }
+  }
+  __syncwarp();
+  // rows 2j and 2j+1 of the strip per step: lanes 0-15 one row, 16-31 the other
+  const int half = lane >> 4, q4 = (lane & 15) * 4;
+  const int n = nbase + q4;
+#pragma unroll 2
+  for (int j = 0; j < 8; j++) {
+    const int lr = 2 * j + half;                 // row inside the warp's strip
+    const int tr = mt * 16 + lr;                 // row inside the tile
+    if (tr < ti.rows && n < p.N) {
+      const int row = tile_row(p.perm, ti, tr);
+      float4 v = *reinterpret_cast<const float4 *>(&so[lr][q4]);
+      float4 *o = reinterpret_cast<float4 *>(p.out + (size_t)row * p.N + n);
+      if (p.accumulate) {
+        const float4 q = *o;
+        v.x = __fadd_rn(q.x, v.x);
+        v.y = __fadd_rn(q.y, v.y);
+        v.z = __fadd_rn(q.z, v.z);
+        v.w = __fadd_rn(q.w, v.w);
       }
-      if (v1 && n0 < p.N) {
-        float2 *o = reinterpret_cast<float2 *>(p.out + (size_t)row1 * p.N + n);
-        float2 v = make_float2(acc[2], acc[3]);
-        if (p.accumulate) {
-          const float2 q = *o;
-          v.x = __fadd_rn(q.x, v.x);
-          v.y = __fadd_rn(q.y, v.y);
-        }
-        __stcs(o, v);
-      }
+      __stcs(o, v);
     }
   }
 }

@@ -43,6 +43,7 @@ namespace bi {
 constexpr int kLeaf = 64;          // k per leaf
 constexpr int kMaxGroupLeaves = 1024;
 constexpr int kMaxSplits = 16;
+constexpr int kMaxBM = 64;         // rows per CTA tile (4 MMA row tiles)
 
 struct ShrinkParams {
   const uint16_t *x;        // [M][K] bf16
@@ -95,7 +96,12 @@ BI_DEV void mma_leaf(float acc[NT][4], const LeafFrag<NT> &f) {
   }
 }
 
-template <int NGW, int MAXD, int PF, bool ASTAGED>
+// PF: leaves of x in flight per thread, in a register ring.  LG: leaves per
+// warp when that count is a power of two known at compile time (the walk is
+// then a binary counter with fixed register slots and a fully unrolled
+// loop); LG = 0 walks any count with the host's post-order schedule on a
+// predicated register stack of MAXD slots.
+template <int NGW, int MAXD, int PF, bool ASTAGED, int LG>
 __global__ void __launch_bounds__(256)
 shrink_kernel(const __grid_constant__ ShrinkParams p) {
   constexpr int NT = NGW / 8;
@@ -103,6 +109,7 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   float *part = reinterpret_cast<float *>(smem_f4);     // [G][BM][r]
   __shared__ TileInfo s_tile;
   __shared__ int32_t s_off[kMaxAdapters + 2];
+  __shared__ int32_t s_rows[kMaxBM];                    // token row of each tile row
 
   const int bm = 16 * p.mtiles;
   const int split = blockIdx.x;
@@ -113,15 +120,22 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   const TileInfo ti = s_tile;
   if (ti.adapter < 0) return;                       // uniform across the cluster
 
+  // e -> (local row, column) of the [bm][r] tile; r is a power of two in
+  // every common configuration, so the split is a shift and a mask
+  const int r_sh = (p.r & (p.r - 1)) == 0 ? __ffs(p.r) - 1 : -1;
+  auto e_row = [&](int e) { return r_sh >= 0 ? e >> r_sh : e / p.r; };
+  auto e_col = [&](int e) { return r_sh >= 0 ? e & (p.r - 1) : e % p.r; };
+
   if (ti.adapter == p.n_ad) {                       // tokens without an adapter
     if (p.mode != BI_SHRINK_ATOMIC && split == 0) {
       for (int e = threadIdx.x; e < ti.rows * p.r; e += blockDim.x) {
-        const int pos = ti.seg_begin + ti.row0 + e / p.r;
-        p.y[(size_t)p.perm[pos] * p.r + e % p.r] = 0.0f;
+        const int pos = ti.seg_begin + ti.row0 + e_row(e);
+        p.y[(size_t)p.perm[pos] * p.r + e_col(e)] = 0.0f;
       }
     }
     return;
   }
+  if ((int)threadIdx.x < ti.rows) s_rows[threadIdx.x] = tile_row(p.perm, ti, threadIdx.x);
 
   // ---- warp role: (leaf group, m-tile, rank group)
   const int per_lg = p.mtiles * p.ngroups;
@@ -142,10 +156,13 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   const int a_stride = p.lc * 128;
   if (a_staged) {
     // A rows [adapter][j][split*lc*64 ...) -> sa[j][...], all threads
-    const int pieces = p.r * p.lc * 8;
+    const int w = p.lc * 8;                          // 16-byte chunks per row
+    const int w_sh = (w & (w - 1)) == 0 ? __ffs(w) - 1 : -1;
+    const int pieces = p.r * w;
     const uint16_t *a0 = p.at + (size_t)ti.adapter * p.r * p.K + (size_t)split * p.lc * kLeaf;
     for (int pc = threadIdx.x; pc < pieces; pc += blockDim.x) {
-      const int j = pc / (p.lc * 8), ch = pc % (p.lc * 8);    // row, 16-byte chunk in the row
+      const int j = w_sh >= 0 ? pc >> w_sh : pc / w;  // row
+      const int ch = pc - j * w;                       // 16-byte chunk in the row
       const int sw = (ch & ~7) | ((ch & 7) ^ ((j & 1) << 2));
       cp_async16(sa + (size_t)j * a_stride + sw * 16, a0 + (size_t)j * p.K + ch * 8);
     }
@@ -157,8 +174,8 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   // the staged slice, or from global memory with the x ones when A is not
   // staged.
   int row0 = 0, row1 = 0;
-  if (v0) row0 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr0] : ti.row0 + lr0;
-  if (v1) row1 = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr1] : ti.row0 + lr1;
+  if (v0) row0 = tile_row(p.perm, ti, lr0);
+  if (v1) row1 = tile_row(p.perm, ti, lr1);
   const uint16_t *xr0 = p.x + (size_t)row0 * p.K + 8 * c;
   const uint16_t *xr1 = p.x + (size_t)row1 * p.K + 8 * c;
   const uint16_t *acol[NT];
@@ -177,18 +194,23 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
     }
   };
   const int swz = (g & 1) << 2;
+  // A fragments of leaf i (index inside the warp's group) from the slice
+  auto a_frags = [&](LeafFrag<NT> &f, int i) {
+    if (a_staged) {
+      const int li = lgi * p.lg + i;               // leaf index inside the CTA's split
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int ch = ((h * 4 + c) ^ swz) << 4;
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+          f.ab[h][t] = *reinterpret_cast<const uint4 *>(sa + (size_t)(ng * NGW + t * 8 + g) * a_stride + li * 128 + ch);
+      }
+    }
+  };
 
   // ---- this warp's leaves: [leaf0, leaf0 + lg), folded in post order
   const int leaf0 = split * p.lc + lgi * p.lg;
-  float st[MAXD][NT][4];
-#pragma unroll
-  for (int d = 0; d < MAXD; d++)
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-#pragma unroll
-      for (int q = 0; q < 4; q++) st[d][t][q] = 0.0f;
-  int depth = 0;
-
+  float res[NT][4];                                // the group's subtree value
   LeafFrag<NT> ring[PF];
 #pragma unroll
   for (int j = 0; j < PF; j++)
@@ -197,57 +219,97 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
     cp_async_wait<0>();                              // this thread's A pieces
     __syncthreads();                                 // everyone's
   }
-  for (int i0 = 0; i0 < p.lg; i0 += PF) {
+
+  if constexpr (LG > 0) {
+    // binary counter: leaf i closes the levels where its index has a 1 bit
+    // (left = the parked subtree, right = the one just finished) and parks
+    // the result at its lowest 0 bit; every index is a compile-time constant
+    constexpr int LOG2 = LG >= 16 ? 4 : (LG >= 8 ? 3 : (LG >= 4 ? 2 : (LG >= 2 ? 1 : 0)));
+    float lv[LOG2 > 0 ? LOG2 : 1][NT][4];
 #pragma unroll
-    for (int j = 0; j < PF; j++) {
-      const int i = i0 + j;
-      if (i < p.lg) {
-        LeafFrag<NT> f = ring[j];
-        if (a_staged) {
-          const int li = lgi * p.lg + i;             // leaf index inside the CTA's split
+    for (int i = 0; i < LG; i++) {
+      LeafFrag<NT> f = ring[i % PF];
+      if (i + PF < LG) load_leaf(ring[i % PF], leaf0 + i + PF);
+      a_frags(f, i);
+      float acc[NT][4];
+      mma_leaf<NT>(acc, f);
 #pragma unroll
-          for (int h = 0; h < 2; h++) {
-            const int ch = ((h * 4 + c) ^ swz) << 4;
-#pragma unroll
-            for (int t = 0; t < NT; t++)
-              f.ab[h][t] = *reinterpret_cast<const uint4 *>(sa + (size_t)(ng * NGW + t * 8 + g) * a_stride + li * 128 + ch);
-          }
-        }
-        if (i + PF < p.lg) load_leaf(ring[j], leaf0 + i + PF);
-        float acc[NT][4];
-        mma_leaf<NT>(acc, f);
-        // push (register stack: every index is a compile-time constant, the
-        // slot is chosen by predication)
-#pragma unroll
-        for (int d = 0; d < MAXD; d++) {
-          const bool hit = d == depth;
+      for (int L = 0; L < LOG2; L++) {
+        if ((i >> L) & 1) {
 #pragma unroll
           for (int t = 0; t < NT; t++)
 #pragma unroll
-            for (int q = 0; q < 4; q++) st[d][t][q] = hit ? acc[t][q] : st[d][t][q];
-        }
-        depth++;
-        // merge the subtrees that end at this leaf: left = st[depth-2]
-        const int nm = p.merges[i];
-#pragma unroll 1
-        for (int m = 0; m < nm; m++) {
+            for (int q = 0; q < 4; q++) acc[t][q] = __fadd_rn(lv[L][t][q], acc[t][q]);
+        } else {
 #pragma unroll
-          for (int d = 1; d < MAXD; d++) {
-            const bool hit = d == depth - 1;
+          for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) lv[L][t][q] = acc[t][q];
+          break;
+        }
+      }
+      if (i == LG - 1)
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+          for (int q = 0; q < 4; q++) res[t][q] = acc[t][q];
+    }
+  } else {
+    float st[MAXD][NT][4];
+#pragma unroll
+    for (int d = 0; d < MAXD; d++)
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) st[d][t][q] = 0.0f;
+    int depth = 0;
+    for (int i0 = 0; i0 < p.lg; i0 += PF) {
+#pragma unroll
+      for (int j = 0; j < PF; j++) {
+        const int i = i0 + j;
+        if (i < p.lg) {
+          LeafFrag<NT> f = ring[j];
+          if (i + PF < p.lg) load_leaf(ring[j], leaf0 + i + PF);
+          a_frags(f, i);
+          float acc[NT][4];
+          mma_leaf<NT>(acc, f);
+          // push (every index is a compile-time constant, the slot is
+          // chosen by predication)
+#pragma unroll
+          for (int d = 0; d < MAXD; d++) {
+            const bool hit = d == depth;
 #pragma unroll
             for (int t = 0; t < NT; t++)
 #pragma unroll
-              for (int q = 0; q < 4; q++) {
-                const float sum = __fadd_rn(st[d - 1][t][q], st[d][t][q]);
-                st[d - 1][t][q] = hit ? sum : st[d - 1][t][q];
-              }
+              for (int q = 0; q < 4; q++) st[d][t][q] = hit ? acc[t][q] : st[d][t][q];
           }
-          depth--;
+          depth++;
+          // merge the subtrees that end at this leaf: left = st[depth-2]
+          const int nm = p.merges[i];
+#pragma unroll 1
+          for (int m = 0; m < nm; m++) {
+#pragma unroll
+            for (int d = 1; d < MAXD; d++) {
+              const bool hit = d == depth - 1;
+#pragma unroll
+              for (int t = 0; t < NT; t++)
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                  const float sum = __fadd_rn(st[d - 1][t][q], st[d][t][q]);
+                  st[d - 1][t][q] = hit ? sum : st[d - 1][t][q];
+                }
+            }
+            depth--;
+          }
         }
       }
     }
+    if (depth != 1) flag_error(p.status, BI_ERR_INVALID_ARG);   // schedule inconsistent
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int q = 0; q < 4; q++) res[t][q] = st[0][t][q];
   }
-  if (depth != 1) flag_error(p.status, BI_ERR_INVALID_ARG);   // schedule inconsistent
 
   // ---- group values -> shared memory, element (local row, column)
   const int E = bm * p.r;
@@ -255,10 +317,8 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   for (int t = 0; t < NT; t++) {
     const int col = ng * NGW + t * 8 + 2 * c;
     float *dst = part + (size_t)lgi * E;
-    dst[lr0 * p.r + col] = st[0][t][0];
-    dst[lr0 * p.r + col + 1] = st[0][t][1];
-    dst[lr1 * p.r + col] = st[0][t][2];
-    dst[lr1 * p.r + col + 1] = st[0][t][3];
+    *reinterpret_cast<float2 *>(dst + lr0 * p.r + col) = make_float2(res[t][0], res[t][1]);
+    *reinterpret_cast<float2 *>(dst + lr1 * p.r + col) = make_float2(res[t][2], res[t][3]);
   }
   __syncthreads();
   // perfect tree over the G groups, in place into group 0
@@ -269,11 +329,7 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
     __syncthreads();
   }
 
-  auto out_index = [&](int e) -> size_t {
-    const int lr = e / p.r;
-    const int row = p.perm ? p.perm[ti.seg_begin + ti.row0 + lr] : ti.row0 + lr;
-    return (size_t)row * p.r + (e % p.r);
-  };
+  auto out_index = [&](int e) -> size_t { return (size_t)s_rows[e_row(e)] * p.r + e_col(e); };
   const int valid_E = ti.rows * p.r;
 
   if (p.mode == BI_SHRINK_ATOMIC) {
@@ -300,10 +356,10 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
 #pragma unroll
     for (int q = 0; q < kMaxSplits; q++) v[q] = q < S ? peer[q][e] : 0.0f;
 #pragma unroll
-    for (int s = 1; s < kMaxSplits; s <<= 1)
+    for (int st = 1; st < kMaxSplits; st <<= 1)
 #pragma unroll
-      for (int q = 0; q + s < kMaxSplits; q += 2 * s)
-        if (q + s < S) v[q] = __fadd_rn(v[q], v[q + s]);
+      for (int q = 0; q + st < kMaxSplits; q += 2 * st)
+        if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
     p.y[out_index(e)] = v[0];
   }
   cluster.sync();   // keep this CTA's shared memory alive until peers are done
@@ -337,10 +393,12 @@ static int tree_merge_schedule(int n, uint8_t *merges) {
   return maxd;
 }
 
-template <int NGW, int MAXD, int PF>
+template <int NGW, int MAXD, int PF, int LG>
 static cudaError_t launch_shrink_t(const ShrinkParams &p, int tiles, int threads, size_t smem,
                                    cudaStream_t stream) {
-  auto kern = p.a_staged ? shrink_kernel<NGW, MAXD, PF, true> : shrink_kernel<NGW, MAXD, PF, false>;
+  void (*kern)(ShrinkParams);
+  if constexpr (PF == 4) kern = shrink_kernel<NGW, MAXD, PF, true, LG>;   // chosen only with A staged
+  else kern = p.a_staged ? shrink_kernel<NGW, MAXD, PF, true, LG> : shrink_kernel<NGW, MAXD, PF, false, LG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -412,10 +470,12 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   const int warps = G * mt * p.ngroups;
   const int threads = 32 * warps;
   const int bm = 16 * mt;
-  const int pf = p.lg >= 2 ? 2 : 1;
   const size_t part_bytes = ((size_t)G * bm * r * sizeof(float) + 127) & ~size_t(127);
   const size_t a_bytes = (size_t)r * p.lc * 128;
   p.a_staged = a_bytes <= 64 * 1024 ? 1 : 0;
+  // x leaves in flight per thread: four when A comes from shared memory
+  // (100 registers, four CTAs per SM), else two (A rides in the ring too)
+  const int pf = p.lg >= 4 && p.a_staged ? 4 : (p.lg >= 2 ? 2 : 1);
   p.a_offset = (int)part_bytes;
   const size_t smem = part_bytes + (p.a_staged ? a_bytes : 0);
   const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
@@ -424,18 +484,22 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
     BI_CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)M * r * sizeof(float), stream));
   }
   cudaError_t e;
-#define BI_SHRINK_PF(NGW_, MAXD_)                                                   \
-  (pf == 2 ? launch_shrink_t<NGW_, MAXD_, 2>(p, tiles, threads, smem, stream)       \
-            : launch_shrink_t<NGW_, MAXD_, 1>(p, tiles, threads, smem, stream))
-  if (ngw == 16) {
-    if (depth <= 4) e = BI_SHRINK_PF(16, 4);
-    else if (depth <= 8) e = BI_SHRINK_PF(16, 8);
-    else e = BI_SHRINK_PF(16, 12);
-  } else {
-    if (depth <= 4) e = BI_SHRINK_PF(8, 4);
-    else if (depth <= 8) e = BI_SHRINK_PF(8, 8);
-    else e = BI_SHRINK_PF(8, 12);
-  }
+  // a power-of-two leaf count per warp up to 16 runs the unrolled counter
+  const int lgc = (p.lg == 1 || p.lg == 2 || p.lg == 4 || p.lg == 8 || p.lg == 16) ? p.lg : 0;
+#define BI_SHRINK_LG(NGW_, PF_)                                                   \
+  (lgc == 1    ? launch_shrink_t<NGW_, 4, PF_, 1>(p, tiles, threads, smem, stream)  \
+   : lgc == 2  ? launch_shrink_t<NGW_, 4, PF_, 2>(p, tiles, threads, smem, stream)  \
+   : lgc == 4  ? launch_shrink_t<NGW_, 4, PF_, 4>(p, tiles, threads, smem, stream)  \
+   : lgc == 8  ? launch_shrink_t<NGW_, 4, PF_, 8>(p, tiles, threads, smem, stream)  \
+   : lgc == 16 ? launch_shrink_t<NGW_, 4, PF_, 16>(p, tiles, threads, smem, stream) \
+   : depth <= 4 ? launch_shrink_t<NGW_, 4, PF_, 0>(p, tiles, threads, smem, stream) \
+   : depth <= 8 ? launch_shrink_t<NGW_, 8, PF_, 0>(p, tiles, threads, smem, stream) \
+                : launch_shrink_t<NGW_, 12, PF_, 0>(p, tiles, threads, smem, stream))
+#define BI_SHRINK_PF(NGW_, MAXD_)                                     \
+  (pf == 4 ? BI_SHRINK_LG(NGW_, 4) : pf == 2 ? BI_SHRINK_LG(NGW_, 2) : BI_SHRINK_LG(NGW_, 1))
+  if (ngw == 16) e = BI_SHRINK_PF(16, 0);
+  else e = BI_SHRINK_PF(8, 0);
+#undef BI_SHRINK_LG
 #undef BI_SHRINK_PF
   return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
