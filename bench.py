@@ -64,7 +64,7 @@ def peaks():
 # --------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling (every 100 ms) of SM clocks and throttle reasons.
+    """nvidia-smi sampling (every 20 ms) of SM clocks and throttle reasons.
     Started before the warm-up; only samples taken inside the timed window
     are summarised (the nearest ones if the window is shorter than one
     sampling period)."""
@@ -82,7 +82,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
