@@ -319,10 +319,10 @@ def run_ours(args, rank, world, device):
         sys.stderr.write(f"kernel {k}: {[round(t * 1e3, 2) for t in v]} us\n")
     per = {k: statistics.median(v) for k, v in per.items()}
     if world > 1:
-        t = torch.tensor([total_ms] + list(per.values()), device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t[0])
-        per = {k: float(t[j + 1]) for j, k in enumerate(per)}
+        from invariant_bi_lora_b200.tp import max_over_ranks
+        t = max_over_ranks([total_ms] + list(per.values()), device="cuda")
+        total_ms = t[0]
+        per = {k: t[j + 1] for j, k in enumerate(per)}
     status = bi.get_device_status(cs)
 
     kern = []

@@ -1,0 +1,92 @@
+"""Tensor-parallel tree GEMM across ranks: the one exchange step of the path.
+
+"Deterministic Inference across Tensor Parallel Sizes That Eliminates
+Training-Inference Mismatch" (Abstract): the intra- and inter-GPU reductions
+follow one hierarchical binary tree, so C = A . W^T has the same bits for
+every TP size.  Row-parallel layout: rank q of `world` holds the contiguous
+K range [q*K/world, (q+1)*K/world) of A and of W (whole 256-wide leaves).
+
+A rank's partial is the canonical tree over its own leaves, which is the
+subtree the single-GPU kernel computes for shard q (`bi_gemm_tree` with
+shards=1 on the rank's slice).  The partials are gathered in rank order
+(all-gather, never an all-reduce, whose order NCCL does not fix) and every
+rank adds the top log2(world) levels with `bi_tree_combine`.  The result is
+bitwise equal to `bi_gemm_tree(A, W, C, shards=world)` on one GPU, and to the
+same call with any other power-of-two shard count.
+
+The compute steps default to the library's kernels; `partial_fn` and
+`combine_fn` exist so that the rank logic can be exercised by CPU process
+groups.
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional
+
+import torch
+import torch.distributed as dist
+
+LEAF = 256
+
+
+def shard_k_range(K: int, world: int, rank: int, leaf: int = LEAF) -> tuple[int, int]:
+    """K range [k0, k1) of `rank`: a contiguous block of whole leaves.
+    world must be a power of two dividing the leaf count."""
+    if K % leaf:
+        raise ValueError(f"K={K} is not a multiple of the leaf width {leaf}")
+    leaves = K // leaf
+    if world < 1 or world & (world - 1) or leaves % world:
+        raise ValueError(f"world={world} must be a power of two dividing {leaves} leaves")
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    per = leaves // world
+    return rank * per * leaf, (rank + 1) * per * leaf
+
+
+def _gpu_partial(A_local, W_local, out):
+    from invariant_bi_lora_b200 import bi
+    bi.gemm_tree(A_local, W_local, out, shards=1)
+
+
+def _gpu_combine(parts, out):
+    from invariant_bi_lora_b200 import bi
+    bi.tree_combine(parts, out)
+
+
+def tree_gemm_tp(A_local: torch.Tensor, W_local: torch.Tensor, C: torch.Tensor,
+                 group: Optional[dist.ProcessGroup] = None,
+                 partial_fn: Optional[Callable] = None,
+                 combine_fn: Optional[Callable] = None) -> torch.Tensor:
+    """C = sum over ranks of A_q . W_q^T, reduced by the canonical tree.
+
+    A_local [M][K/world] and W_local [N][K/world] (bf16, K-contiguous) are
+    this rank's slices; C [M][N] fp32 receives the full result on every
+    rank.  Collective: every rank of `group` must call it with the same M, N
+    and slice width."""
+    partial_fn = partial_fn or _gpu_partial
+    combine_fn = combine_fn or _gpu_combine
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world & (world - 1):
+        raise ValueError(f"world size {world} is not a power of two")
+    M, N = C.shape
+    if A_local.shape[0] != M or W_local.shape[0] != N or A_local.shape[1] != W_local.shape[1]:
+        raise ValueError("slice shapes do not match C")
+    if world == 1:
+        partial_fn(A_local, W_local, C)
+        return C
+    partial = torch.empty(M, N, dtype=torch.float32, device=C.device)
+    partial_fn(A_local, W_local, partial)
+    parts = torch.empty(world * M, N, dtype=torch.float32, device=C.device)
+    dist.all_gather_into_tensor(parts, partial, group=group)      # concatenated in rank order
+    combine_fn(parts.view(world, M, N), C)
+    return C
+
+
+def max_over_ranks(values, device="cpu", group: Optional[dist.ProcessGroup] = None) -> list[float]:
+    """Elementwise maximum of `values` over the ranks of `group` (one
+    all-reduce); the values themselves when no process group is running."""
+    vals = [float(v) for v in values]
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return [float(v) for v in t.tolist()]
