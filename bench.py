@@ -256,6 +256,16 @@ def run_ours(args, rank, world, device):
     # everything below runs with cs as the current stream: graph replays go to
     # the current stream, and the timing events must be on the same one
     cs.wait_stream(torch.cuda.current_stream())
+    if args.eager_only:
+        # profiler launch lists: the same kernels launched eagerly, no graphs,
+        # no timing (ncu's replay of graph nodes does not take the cluster
+        # launches here)
+        with torch.cuda.stream(cs):
+            for _ in range(args.warmup + args.steps):
+                step_body()
+            torch.cuda.synchronize()
+        return {"note": "eager launches for a profiler launch list; not a measurement",
+                "steps": args.steps, "warmup": args.warmup, "status": bi.get_device_status(cs)}
     with torch.cuda.stream(cs):
         # eager warm-up (TMA descriptors, kernel attributes, occupancy queries)
         for _ in range(args.warmup):
@@ -492,6 +502,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--eager-only", action="store_true",
+                    help="launch the step's kernels eagerly and exit (for ncu launch lists)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -507,7 +519,7 @@ def main():
         return
 
     # CPU baseline first (rank 0, N=1 only), before any GPU work.
-    cpu = cpu_baseline_entry(args.cpu_seconds) if (rank == 0 and world == 1) else None
+    cpu = cpu_baseline_entry(args.cpu_seconds) if (rank == 0 and world == 1 and not args.eager_only) else None
 
     torch.cuda.set_device(local)
     if world > 1:

@@ -211,7 +211,10 @@ BI_DEV float max4(float m, float4 v) {
   return b;
 }
 
-__global__ void __launch_bounds__(1024)
+// THREADS = 4096 / C.  The minimum-blocks bound keeps the 256-thread form
+// (C = 16) at <= 48 registers, so five CTAs (smem-limited) share an SM.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, THREADS == 256 ? 5 : 0)
 log_softmax_kernel(const __grid_constant__ LsmParams p) {
   extern __shared__ float4 lsm_smem[];
   __shared__ float s_red[32];
@@ -374,26 +377,33 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
   p.C = C;
   const size_t smem = (size_t)p.J * (bi::kLsmT / C) * 16;
   if (smem > 200 * 1024) return BI_ERR_UNSUPPORTED_SHAPE;
-  cudaError_t e = cudaFuncSetAttribute(bi::log_softmax_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return BI_ERR_CUDA;
-  if (C > 8) {
-    e = cudaFuncSetAttribute(bi::log_softmax_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return BI_ERR_CUDA;
+  auto launch = [&](auto kern) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (C > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)rows * C, 1, 1);
+    cfg.blockDim = dim3(bi::kLsmT / C, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  };
+  cudaError_t e;
+  switch (C) {
+    case 4: e = launch(bi::log_softmax_kernel<1024>); break;
+    case 8: e = launch(bi::log_softmax_kernel<512>); break;
+    default: e = launch(bi::log_softmax_kernel<256>); break;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)rows * C, 1, 1);
-  cfg.blockDim = dim3(bi::kLsmT / C, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, bi::log_softmax_kernel, p);
   return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
