@@ -88,11 +88,14 @@ def test_log_softmax_shapes(n):
     assert np.array_equal(lsm(x), oracle.log_softmax_canon(x).view(np.uint32))
 
 
-def test_log_softmax_wide_range_rows():
+@pytest.mark.parametrize("R", [7, 160])
+def test_log_softmax_wide_range_rows(R):
     """Logits spread over hundreds: many vectors take the general exp path
-    (x - max < -87, down to the flush to zero below -103)."""
-    x = synth.normal_f32((7, 151936), 60.0, seed=77)
+    (x - max < -87, down to the flush to zero below -103), in a few rows
+    and in enough rows for several waves of clusters."""
+    x = synth.normal_f32((R, 151936), 60.0, seed=77)
     x[3, ::5] = -1e4
+    x[R - 1, 7::3] = -1e4
     assert np.array_equal(lsm(x), oracle.log_softmax_canon(x).view(np.uint32))
 
 
