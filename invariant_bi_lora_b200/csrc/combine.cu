@@ -65,6 +65,31 @@ tree_combine_kernel(const __grid_constant__ CombineParams p) {
   }
 }
 
+// s = S, a power of two: the canonical tree is the perfect tree, so all S
+// loads of a thread are issued together and added pairwise afterwards (the
+// general kernel's loop issues one load per merge step and waits on each).
+template <int S>
+__global__ void __launch_bounds__(256)
+tree_combine_pow2_kernel(const float *__restrict__ parts, float *__restrict__ out, size_t nv) {
+  const float4 *src = reinterpret_cast<const float4 *>(parts);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 v[S];
+#pragma unroll
+    for (int j = 0; j < S; j++) v[j] = __ldcs(src + (size_t)j * nv + i);
+#pragma unroll
+    for (int st = 1; st < S; st <<= 1)
+#pragma unroll
+      for (int q = 0; q + st < S; q += 2 * st) {
+        v[q].x = __fadd_rn(v[q].x, v[q + st].x);
+        v[q].y = __fadd_rn(v[q].y, v[q + st].y);
+        v[q].z = __fadd_rn(v[q].z, v[q + st].z);
+        v[q].w = __fadd_rn(v[q].w, v[q + st].w);
+      }
+    __stcs(reinterpret_cast<float4 *>(out) + i, v[0]);
+  }
+}
+
 // Post-order merge schedule of the canonical halving tree over n leaves.
 void tree_schedule(int n, uint8_t *merges) {
   std::fill(merges, merges + n, 0);
@@ -94,7 +119,13 @@ bi_status tree_combine_launch(const float *partials, float *out, int s, size_t c
   tree_schedule(s, p.merges);
   const size_t nv = count / 4;
   const unsigned blocks = (unsigned)std::min<size_t>((nv + 255) / 256, 148 * 8);
-  tree_combine_kernel<<<blocks, 256, 0, stream>>>(p);
+  switch (s) {
+    case 2: tree_combine_pow2_kernel<2><<<blocks, 256, 0, stream>>>(partials, out, nv); break;
+    case 4: tree_combine_pow2_kernel<4><<<blocks, 256, 0, stream>>>(partials, out, nv); break;
+    case 8: tree_combine_pow2_kernel<8><<<blocks, 256, 0, stream>>>(partials, out, nv); break;
+    case 16: tree_combine_pow2_kernel<16><<<blocks, 256, 0, stream>>>(partials, out, nv); break;
+    default: tree_combine_kernel<<<blocks, 256, 0, stream>>>(p); break;
+  }
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

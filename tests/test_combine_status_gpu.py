@@ -13,7 +13,7 @@ from invariant_bi_lora_b200 import bi, synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("s,count", [(1, 16), (2, 4096), (3, 1000), (5, 4), (8, 1 << 20), (64, 4096), (6, 0)])
+@pytest.mark.parametrize("s,count", [(1, 16), (2, 4096), (3, 1000), (4, 4100), (5, 4), (8, 1 << 20), (16, 65540), (64, 4096), (6, 0)])
 def test_tree_combine(s, count):
     g = np.random.default_rng(s)
     parts = (g.standard_normal((s, count)) * g.choice([1e8, 1.0, 1e-3, 3.5], size=(s, count))).astype(np.float32)
