@@ -24,11 +24,14 @@ namespace bi {
 
 // ======================================================================
 // RMSNorm: T = 512 lanes of V = 8 bf16.  One CTA of THREADS threads per
-// row; thread u owns the LPT = 512/THREADS adjacent lanes u*LPT .. +LPT-1
-// (a subtree of the lane tree), so it reads LPT*16 contiguous bytes per
-// step.  The row stays in registers (VPL vectors per lane) between the sum
-// and the scaling, so x is read from HBM once.  128 threads per row keep 16
-// rows (128 KB) in flight per SM.
+// row; thread u owns the LPT = 512/THREADS lanes u + THREADS*s (slot s), so
+// each load or store instruction of a warp covers 32 consecutive vectors
+// (512 contiguous bytes).  Slot s of all threads is the lane block
+// [THREADS*s, THREADS*(s+1)), a subtree of the lane tree: a warp's 32 lanes
+// of a slot are added by the xor butterfly, and the 16 (slot, warp) values
+// -- in lane order -- by a perfect tree that every warp evaluates itself.
+// The row stays in registers (VPL vectors per lane) between the sum and the
+// scaling, so x is read from HBM once.
 // ======================================================================
 constexpr int kNormT = 512;
 
@@ -38,12 +41,14 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
                uint16_t *__restrict__ y, int n, float eps) {
   constexpr int LPT = kNormT / THREADS;
   constexpr int NW = THREADS / 32;
-  __shared__ float s_warp[NW];
-  __shared__ float s_inv;
+  static_assert(LPT * NW == kNormT / 32, "16 (slot, warp) groups");
+  __shared__ float s_grp[kNormT / 32];          // index s * NW + warp
   const int u = threadIdx.x;
+  const int lane = u & 31, warp = u >> 5;
   const size_t row = blockIdx.x;
   const int nvec = n / 8;
   const uint16_t *xr = x + row * n;
+  auto vidx = [&](int j, int sl) { return j * kNormT + sl * THREADS + u; };
 
   uint4 v[VPL][LPT];
   // small rows: w is fetched with x, so the scaling pass does not wait on
@@ -57,7 +62,7 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
   for (int j = 0; j < VPL; j++)
 #pragma unroll
     for (int l = 0; l < LPT; l++) {
-      const int vi = j * kNormT + u * LPT + l;
+      const int vi = vidx(j, l);
       v[j][l] = vi < nvec ? ldg128_stream(xr + 8 * vi) : make_uint4(0, 0, 0, 0);
       if constexpr (PREW) wv_pre[j][l] = vi < nvec ? ldg128(w + 8 * vi) : make_uint4(0, 0, 0, 0);
     }
@@ -65,7 +70,7 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
   for (int j = 0; j < VPL; j++)
 #pragma unroll
     for (int l = 0; l < LPT; l++) {
-      if (j * kNormT + u * LPT + l < nvec) {
+      if (vidx(j, l) < nvec) {
         const uint32_t q[4] = {v[j][l].x, v[j][l].y, v[j][l].z, v[j][l].w};
 #pragma unroll
         for (int e = 0; e < 4; e++) {
@@ -75,42 +80,36 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
         }
       }
     }
-  // perfect tree over this thread's LPT adjacent lanes
+  // each slot: the warp's 32 lanes by the butterfly
 #pragma unroll
-  for (int st = 1; st < LPT; st <<= 1)
-#pragma unroll
-    for (int l = 0; l + st < LPT; l += 2 * st) p[l] = __fadd_rn(p[l], p[l + st]);
-  float sum = warp_tree_sum(p[0]);
-  if ((u & 31) == 0) s_warp[u >> 5] = sum;
-  __syncthreads();
-  if (u < 32) {
-    float q = u < NW ? s_warp[u] : 0.0f;
-#pragma unroll
-    for (int o = 1; o < NW; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
-    if (u == 0) {
-      const float ms = __fdiv_rn(q, (float)n);
-      s_inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-    }
+  for (int l = 0; l < LPT; l++) {
+    const float sv = warp_tree_sum(p[l]);
+    if (lane == 0) s_grp[l * NW + warp] = sv;
   }
   __syncthreads();
-  const float inv = s_inv;
+  // the 16 group values in lane order, perfect tree on lanes 0..15
+  float q = lane < kNormT / 32 ? s_grp[lane] : 0.0f;
+#pragma unroll
+  for (int o = 1; o < kNormT / 32; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+  q = __shfl_sync(0xffffffffu, q, 0);
+  const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(q, (float)n), eps)));
   uint16_t *yr = y + row * n;
 #pragma unroll
   for (int j = 0; j < VPL; j++)
 #pragma unroll
     for (int l = 0; l < LPT; l++) {
-      const int vi = j * kNormT + u * LPT + l;
+      const int vi = vidx(j, l);
       if (vi < nvec) {
         uint4 wv;
         if constexpr (PREW) wv = wv_pre[PREW ? j : 0][l];
         else wv = ldg128(w + 8 * vi);
-        const uint32_t q[4] = {v[j][l].x, v[j][l].y, v[j][l].z, v[j][l].w};
+        const uint32_t q4[4] = {v[j][l].x, v[j][l].y, v[j][l].z, v[j][l].w};
         const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; e++) {
-          const float lo = __fmul_rn(__fmul_rn(bf16lo(q[e]), inv), bf16lo(wq[e]));
-          const float hi = __fmul_rn(__fmul_rn(bf16hi(q[e]), inv), bf16hi(wq[e]));
+          const float lo = __fmul_rn(__fmul_rn(bf16lo(q4[e]), inv), bf16lo(wq[e]));
+          const float hi = __fmul_rn(__fmul_rn(bf16hi(q4[e]), inv), bf16hi(wq[e]));
           o[e] = pack_bf16x2(lo, hi);
         }
         *reinterpret_cast<uint4 *>(yr + 8 * vi) = make_uint4(o[0], o[1], o[2], o[3]);

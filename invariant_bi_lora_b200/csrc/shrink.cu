@@ -462,6 +462,10 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   while (p.lc / G > 8 && p.lc % (G * 2) == 0 && G * 2 * p.ngroups <= 8) G *= 2;
   int mt = std::min(4, (M + 15) / 16);
   while (mt > 1 && mt * G * p.ngroups > 8) mt >>= 1;
+  // one row tile of 16 (decode-sized M): spend the CTA's eight warps on
+  // leaf groups instead, so that every leaf's loads leave at once
+  if (mt == 1)
+    while (p.lc % (G * 2) == 0 && G * 2 * p.ngroups <= 8) G *= 2;
   p.mtiles = mt;
   p.groups = G;
   p.lg = p.lc / G;
