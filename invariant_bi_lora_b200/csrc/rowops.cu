@@ -119,16 +119,20 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
 
 // ======================================================================
 // mean: T = 1024 lanes of V = 4 fp32.  One CTA of 256 threads per row;
-// thread u owns the four adjacent lanes 4u..4u+3 (a subtree of the lane
-// tree), so each step it reads 64 contiguous bytes.
+// thread u owns the four lanes u + 256*s (slot s), so each load of a warp
+// covers 512 contiguous bytes.  Slot s is the lane block [256s, 256s+256),
+// a subtree: a warp's 32 lanes of a slot by the xor butterfly, then the 32
+// (slot, warp) values in lane order by a perfect tree in one warp.
 // ======================================================================
 constexpr int kLaneT = 1024;
 constexpr int kMeanThreads = 256;
 
 __global__ void __launch_bounds__(kMeanThreads)
 mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
-  __shared__ float s_warp[kMeanThreads / 32];
+  constexpr int NW = kMeanThreads / 32;
+  __shared__ float s_grp[kLaneT / 32];           // index s * NW + warp
   const int u = threadIdx.x;
+  const int lane = u & 31, warp = u >> 5;
   const size_t row = blockIdx.x;
   const int nvec = n / 4;
   const float4 *xr = reinterpret_cast<const float4 *>(x + row * n);
@@ -136,28 +140,28 @@ mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
   for (int base = 0; base < nvec; base += kLaneT) {
     float4 v[4];
 #pragma unroll
-    for (int l = 0; l < 4; l++) {
-      const int vi = base + 4 * u + l;
-      v[l] = vi < nvec ? __ldcs(xr + vi) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < 4; s++) {
+      const int vi = base + s * kMeanThreads + u;
+      v[s] = vi < nvec ? __ldcs(xr + vi) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int l = 0; l < 4; l++) {
-      if (base + 4 * u + l < nvec) {
-        p[l] = __fadd_rn(p[l], v[l].x);
-        p[l] = __fadd_rn(p[l], v[l].y);
-        p[l] = __fadd_rn(p[l], v[l].z);
-        p[l] = __fadd_rn(p[l], v[l].w);
+    for (int s = 0; s < 4; s++) {
+      if (base + s * kMeanThreads + u < nvec) {
+        p[s] = __fadd_rn(p[s], v[s].x);
+        p[s] = __fadd_rn(p[s], v[s].y);
+        p[s] = __fadd_rn(p[s], v[s].z);
+        p[s] = __fadd_rn(p[s], v[s].w);
       }
     }
   }
-  float s = __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
-  s = warp_tree_sum(s);
-  if ((u & 31) == 0) s_warp[u >> 5] = s;
+#pragma unroll
+  for (int s = 0; s < 4; s++) {
+    const float sv = warp_tree_sum(p[s]);
+    if (lane == 0) s_grp[s * NW + warp] = sv;
+  }
   __syncthreads();
   if (u < 32) {
-    float q = u < kMeanThreads / 32 ? s_warp[u] : 0.0f;
-#pragma unroll
-    for (int o = 1; o < kMeanThreads / 32; o <<= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+    const float q = warp_tree_sum(s_grp[lane]);
     if (u == 0) out[row] = __fdiv_rn(q, (float)n);
   }
 }
