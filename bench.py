@@ -225,6 +225,12 @@ class Workload:
 
 KERNEL_REPS = 10      # reps per kernel graph in the per-kernel timing block
 
+# DRAM bytes (read + write) of one launch, from an ncu capture of the same
+# kernel and workload (dram__bytes_read.sum + dram__bytes_write.sum; see
+# profiles/log_softmax_rows256_v151936.md for the command).  Only kernels
+# unchanged since their capture are listed.
+MEASURED_TRAFFIC = {"log_softmax": 2489417216 + 2431791616}
+
 
 def capture(fn, stream):
     """Capture fn() into a CUDA graph on `stream`."""
@@ -312,18 +318,21 @@ def run_ours(args, rank, world, device):
         clocks.mark(h0, h1)
         total_ms = t0.elapsed_time(t1)
 
-        # ---------------- per-kernel durations: (R x [flush, kernel]) - (R x [flush])
-        per = {name: [] for (name, *_r) in wl.kernels}
-        for _ in range(3):
+        # ---------------- per-kernel durations: (R x [flush, kernel]) - (R x [flush]),
+        # the flush-only graph timed right before and right after each kernel
+        # graph (their mean is subtracted), five rounds, median
+        def replay_ms(g):
             a, b = ev(), ev()
-            a.record(cs); g_flush.replay(); b.record(cs)
+            a.record(cs); g.replay(); b.record(cs)
             torch.cuda.synchronize()
-            tf = a.elapsed_time(b)
+            return a.elapsed_time(b)
+        per = {name: [] for (name, *_r) in wl.kernels}
+        for _ in range(5):
             for (name, *_r), g in zip(wl.kernels, g_kern):
-                a, b = ev(), ev()
-                a.record(cs); g.replay(); b.record(cs)
-                torch.cuda.synchronize()
-                per[name].append(max(a.elapsed_time(b) - tf, 1e-6) / R)
+                f0 = replay_ms(g_flush)
+                tk = replay_ms(g)
+                f1 = replay_ms(g_flush)
+                per[name].append(max(tk - 0.5 * (f0 + f1), 1e-6) / R)
         clk = clocks.stop()
     for k, v in per.items():
         sys.stderr.write(f"kernel {k}: {[round(t * 1e3, 2) for t in v]} us\n")
@@ -365,10 +374,11 @@ def run_ours(args, rank, world, device):
                    "parallelism": f"dp{world} (independent replicas, no collective)",
                    "l2": "flushed before every kernel (256 MiB written, then read back: cold, clean L2)",
                    "timing": "step = one CUDA-graph replay of the whole path; per-kernel time = "
-                             f"(graph of {R} x [flush, kernel]) - (graph of {R} x [flush]), CUDA events"},
+                             f"(graph of {R} x [flush, kernel]) - mean of the (graph of {R} x [flush]) "
+                             "replays just before and after it, CUDA events, median of 5"},
         "roofline": {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"],
                      "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
-                     "traffic": None, "peak_source": pk["source"]},
+                     "traffic": MEASURED_TRAFFIC.get(dom["name"]), "peak_source": pk["source"]},
         "shrink_roofline": {"bound": "hbm", "achieved": tree["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                             "frac": tree["frac"], "bytes_per_launch": SHRINK_BYTES},
         "delta_vs_atomic_pct": round(100.0 * (tree["us"] / by["shrink_atomic_s8"]["us"] - 1.0), 2),
