@@ -62,8 +62,8 @@ struct ShrinkParams {
   int mode;
   int a_staged;             // 1: the CTA's A slice sits in shared memory
   int a_offset;             // bytes from the start of dynamic shared memory to the A slice
-  int g_offset;             // bytes to the gather slots (mode TREE: the other ranks' partials, in rank 0)
-  int push;                 // mode TREE: 1 = partials pushed to rank 0, 0 = every rank pulls a share
+  int g_offset;             // bytes to the exchange slots (mode TREE)
+  int gather0;              // mode TREE: 1 = all partials to rank 0, 0 = reduce-scatter over the ranks
   uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
 };
 
@@ -344,17 +344,20 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   }
 
   // ---- mode TREE: the splits CTAs of this tile form one cluster; rank q
-  // holds the subtree of leaves [q*lc, (q+1)*lc); the S partials meet by the
-  // perfect tree over the ranks.
+  // holds the subtree of leaves [q*lc, (q+1)*lc).  The tile's E elements
+  // are cut into S shares; rank q finishes share q.  Before one cluster
+  // barrier every rank stores share t of its partial into rank t's slot
+  // [q] through distributed shared memory (a reduce-scatter by pushes);
+  // after it (release / acquire) each rank adds the S values of its share
+  // by the perfect tree over the ranks, from its own shared memory, and
+  // writes y.  Nothing reads a peer's memory after the barrier, so one
+  // barrier is enough, and every SM receives only (S-1)/S of one partial.
   cg::cluster_group cluster = cg::this_cluster();
   const int S = p.splits;
-  if (p.push) {
-    // Ranks 1..S-1 store their partial into rank 0's gather slots through
-    // distributed shared memory, then one cluster barrier (release /
-    // acquire) publishes them; rank 0 adds the partials from its own shared
-    // memory and writes y, the others exit.  Nothing reads a peer's memory
-    // after the barrier, so one barrier is enough.
-    float *gslots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);  // [S-1][E]
+  if (p.gather0) {
+    // small tiles: ranks 1..S-1 push their whole partial into rank 0's
+    // slots [S-1][E]; after the barrier rank 0 alone adds and writes y
+    float *gslots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);
     if (split != 0) {
       float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(gslots, 0) + (size_t)(split - 1) * E);
       const float4 *src = reinterpret_cast<const float4 *>(part);
@@ -377,17 +380,23 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
     }
     return;
   }
-  // Partials too large to gather in one CTA: each CTA finishes a strided
-  // share of the elements, reading the ranks' partials where they are.
-  cluster.sync();
-  const float *peer[kMaxSplits];
-#pragma unroll
-  for (int q = 0; q < kMaxSplits; q++)
-    peer[q] = q < S ? cluster.map_shared_rank(part, q) : part;
-  for (int e = split * blockDim.x + threadIdx.x; e < valid_E; e += S * blockDim.x) {
+  const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
+  float *slots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);  // [S][share]
+  for (int t = 0; t < S; t++) {
+    if (t == split) continue;
+    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
+    const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
+    for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  for (int i = threadIdx.x; i < share; i += blockDim.x) {
+    const int e = split * share + i;
+    if (e >= valid_E) break;
     float v[kMaxSplits];
 #pragma unroll
-    for (int q = 0; q < kMaxSplits; q++) v[q] = q < S ? peer[q][e] : 0.0f;
+    for (int q = 0; q < kMaxSplits; q++)
+      v[q] = q < S ? (q == split ? part[e] : slots[(size_t)q * share + i]) : 0.0f;
 #pragma unroll
     for (int st = 1; st < kMaxSplits; st <<= 1)
 #pragma unroll
@@ -395,7 +404,6 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
         if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
     p.y[out_index(e)] = v[0];
   }
-  cluster.sync();   // keep this CTA's shared memory alive until peers are done
 }
 
 // ----------------------------------------------------------------------
@@ -514,16 +522,16 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   // (100 registers, four CTAs per SM), else two (A rides in the ring too)
   const int pf = p.lg >= 4 && p.a_staged ? 4 : (p.lg >= 2 ? 2 : 1);
   p.a_offset = (int)part_bytes;
-  // mode TREE gathers the partials in rank 0 when they are small (one
-  // 16-row tile: 1 KB per rank at r = 16).  Measured: 3.9 -> 2.7 us at
-  // M = 16, but 11.8 -> 19 us for 64-row tiles (28 KB gathered per
-  // cluster), where every rank pulling a share is faster.
-  size_t gather_bytes = mode == BI_SHRINK_TREE && splits > 1 ? (size_t)(splits - 1) * bm * r * sizeof(float) : 0;
+  // mode TREE exchange slots: one partial's worth (S shares of E/S) for the
+  // reduce-scatter; S-1 partials in rank 0 for small tiles (<= 8 KB in all),
+  // where one CTA adding everything beats spreading it (M = 16: 2.8 us
+  // against 4.8 us; at 64-row tiles the rank-0 gather took 19 us)
+  const size_t part1 = (size_t)bm * r * sizeof(float);
+  p.gather0 = mode == BI_SHRINK_TREE && splits > 1 && (size_t)(splits - 1) * part1 <= 8 * 1024 ? 1 : 0;
+  const size_t slot_bytes = mode == BI_SHRINK_TREE && splits > 1 ? (p.gather0 ? (size_t)(splits - 1) * part1 : part1) : 0;
   const size_t base_smem = part_bytes + (p.a_staged ? a_bytes : 0);
-  p.push = gather_bytes > 0 && gather_bytes <= 8 * 1024 ? 1 : 0;
-  if (!p.push) gather_bytes = 0;
   p.g_offset = (int)base_smem;
-  const size_t smem = base_smem + gather_bytes;
+  const size_t smem = base_smem + slot_bytes;
   const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
 
   if (mode == BI_SHRINK_ATOMIC) {
