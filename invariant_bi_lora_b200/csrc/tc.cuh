@@ -1,5 +1,5 @@
 // tc.cuh -- sm_100a building blocks: mbarriers with bounded waits, TMA tile
-// loads (no multicast), tcgen05 MMA / TMEM allocation / TMEM loads and
+// loads into this CTA only, tcgen05 MMA / TMEM allocation / TMEM loads and
 // stores, and the UMMA shared-memory and instruction descriptors.
 //
 // Descriptor layouts (PTX ISA, tcgen05 "shared memory descriptor" and
@@ -71,7 +71,7 @@ BI_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
 
 // ------------------------------------------------------------------ TMA
 // 2-D tile load into shared memory, completion counted on `bar` (bytes).
-// No multicast.  x (innermost, elements) must be a multiple of 8 for bf16.
+// This CTA only.  x (innermost, elements) must be a multiple of 8 for bf16.
 BI_DEV void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
@@ -80,7 +80,7 @@ BI_DEV void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x,
       : "memory");
 }
 // Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple
-// of 16), completion counted on `bar` (bytes).  No multicast.
+// of 16), completion counted on `bar` (bytes).  This CTA only.
 BI_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
