@@ -364,6 +364,7 @@ def run_ours(args, rank, world, device):
     gemm = by.get("gemm")
     e2e = measure_e2e(wl, bi, args) if rank == 0 else None
     atomic_var = atomic_variation(wl, bi) if rank == 0 else None
+    stream16 = shrink16_stream(wl, bi, pk) if rank == 0 else None
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -385,6 +386,7 @@ def run_ours(args, rank, world, device):
         "speedup_vs_unsplit_pct": round(100.0 * (by["shrink_unsplit"]["us"] / tree["us"] - 1.0), 2),
         "bi_gemm_tflops": None if gemm is None else gemm["tflops"],
         "atomic_variation": atomic_var,
+        "shrink16_cold_stream": stream16,
         "kernels": kern,
         "kernel_sum_ms": round(sum(per.values()), 4),
         "gpu_launches": args.steps * sum(k["launches"] for k in kern),
@@ -416,6 +418,41 @@ def atomic_variation(wl, bi, replays=100):
         out[mode] = {"replays": replays, "distinct_outputs": uniq,
                      "pairs_differing": round(pairs_diff / npairs, 4),
                      "elements_differing_vs_first": round(float(np.mean(h[1:] != h[0])), 4)}
+    return out
+
+
+def shrink16_stream(wl, bi, pk, l2_bytes=126 << 20):
+    """The M=16 shrink as a cold stream: back-to-back calls in one CUDA graph,
+    each on its own copy of x and A, the copies together three times the L2
+    size, so every call reads from DRAM.  Per-call time (median of 5 graph
+    replays / calls) and its HBM fraction; latency, not bandwidth, bounds a
+    263 KB call.  Outside the timed region."""
+    call_bytes = 16 * 4096 * 2 * 2 + 16 * 16 * 4
+    copies = -(-3 * l2_bytes // call_bytes)
+    xs = wl.x16.unsqueeze(0).expand(copies, -1, -1).contiguous()
+    As = wl.A16.unsqueeze(0).expand(copies, -1, -1).contiguous()
+    out = {"calls": copies, "bytes_per_call": call_bytes}
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        for mode, splits in (("tree", 8), ("atomic", 8), ("unsplit", 1)):
+            bi.lora_shrink(xs[0], As[0], wl.y16, splits, mode)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                for i in range(copies):
+                    bi.lora_shrink(xs[i], As[i], wl.y16, splits, mode)
+            ts = []
+            for _ in range(5):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st); g.replay(); b.record(st)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) * 1e3 / copies)
+            us = statistics.median(ts)
+            gbs = call_bytes / us / 1e3
+            out[mode] = {"us_per_call": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4)}
+            del g
+    del xs, As
     return out
 
 
