@@ -74,7 +74,7 @@ BI_DEV float bi_exp_fast(float x) {
   return __fmul_rn(p, __int_as_float((ni + 127) << 23));
 }
 
-// Two lanes at once: sm_100's packed fp32 instructions (add/sub/mul/fma
+// Two lanes at once: sm_100's packed fp32 instructions (sub/mul/fma
 // .rn.f32x2) round each lane exactly as the scalar instruction does, so
 // bi_exp_fast2 gives bi_exp_fast's bits for both lanes in about half the
 // issued instructions.  fma(-n, c, r) is computed as fma(n, -c, r): the
@@ -92,11 +92,6 @@ BI_DEV float2 upk2(uint64_t r) {
 BI_DEV uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-BI_DEV uint64_t add2_rn(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 BI_DEV uint64_t sub2_rn(uint64_t a, uint64_t b) {

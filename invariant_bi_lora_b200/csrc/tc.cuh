@@ -79,15 +79,6 @@ BI_DEV void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x,
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple
-// of 16), completion counted on `bar` (bytes).  This CTA only.
-BI_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 // Per-thread 16-byte asynchronous copy global -> shared (LDGSTS, L2 only),
 // and an arrival on `bar` that fires once all of this thread's earlier
 // cp.async copies have landed (the barrier's count must include it: noinc).
@@ -98,9 +89,6 @@ BI_DEV void cp_async16(void *dst, const void *src) {
 BI_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 BI_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-BI_DEV void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 BI_DEV void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
