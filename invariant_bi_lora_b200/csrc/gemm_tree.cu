@@ -20,9 +20,10 @@
 // 2..9 fold finished leaves into the pending stack of the post-order tree
 // walk; each epilogue thread owns one row (its TMEM lane) and half of the
 // tile's columns.  Two layouts:
-//  * BN = 128, 1/2/4/8 leaves per shard (known at compile time): the walk is
-//    a binary counter; level 0 of the pending stack sits in registers,
-//    levels 1 and 2 in TMEM (2 x 128 buffer + 2 x 128 stack = 512 columns).
+//  * BN = 128, 1/2/4/8/16 leaves per shard (known at compile time): the walk
+//    is a binary counter; level 0 of the pending stack sits in registers,
+//    the higher levels in TMEM (2 x 128 leaf buffers + 2 x 128 stack, or for
+//    16 leaves 1 x 128 buffer + 3 x 128 stack: 512 columns either way).
 //    The wide tile halves the operand bytes per flop that L2 must deliver.
 //  * BN = 64, any leaf count up to 64: the host-computed post-order schedule
 //    (merges per leaf), stack of 6 slots in TMEM (2 x 64 + 6 x 64 columns).
@@ -75,7 +76,7 @@ BI_DEV void add_rn(float (&cur)[N], const float (&left)[N]) {
   for (int q = 0; q < N; q++) cur[q] = __fadd_rn(left[q], cur[q]);
 }
 
-// LPS = 0: BN = 64, any leaf count (p.merges).  LPS = 1, 2, 4, 8: BN = 128.
+// LPS = 0: BN = 64, any leaf count (p.merges).  LPS = 1, 2, 4, 8, 16: BN = 128.
 template <int BN, int LPS>
 __global__ void __launch_bounds__(tg::THREADS, 1)
 gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
@@ -87,7 +88,10 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
   static_assert(LPS == 0 || BN == 128, "counter layout is the 128-wide tile");
   static_assert(LPS != 0 || BN == 64, "schedule layout is the 64-wide tile");
-  constexpr int LOG2 = LPS >= 8 ? 3 : (LPS >= 4 ? 2 : (LPS >= 2 ? 1 : 0));
+  constexpr int LOG2 = LPS >= 16 ? 4 : (LPS >= 8 ? 3 : (LPS >= 4 ? 2 : (LPS >= 2 ? 1 : 0)));
+  // TMEM leaf buffers: two, except for 16 leaves, whose three TMEM levels
+  // (128 columns each) leave room for one
+  constexpr int NBUF = LPS == 16 ? 1 : 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sa = smem;
@@ -184,7 +188,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
           umma_commit(&tail->tfull[buf]);
-          if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+          if (++buf == NBUF) { buf = 0; buf_phase ^= 1; }
         }
       }
     }
@@ -215,7 +219,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->tempty[buf]);
-        if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+        if (++buf == NBUF) { buf = 0; buf_phase ^= 1; }
         // subtrees that end at this leaf: cur = left + cur, left popped
         for (int m = p.merges[leaf]; m > 0; m--) {
           top--;
@@ -245,8 +249,8 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ---------------- epilogue: binary counter over LPS leaves.  Leaf i
     // closes the subtrees of the levels where its index has a 1 bit (left =
     // the waiting subtree, right = the one just finished); at its lowest 0
-    // bit it parks the result.  Level 0 parks in registers, levels 1 and 2
-    // in TMEM columns 256 and 384.
+    // bit it parks the result.  Level 0 parks in registers, level L >= 1 in
+    // TMEM columns from (NBUF + L - 1) * 128.
     const int ew = warp - 2;
     const int quad = warp & 3;                  // TMEM lane quadrant of this warp
     const int half = ew >> 2;                   // which 64 of the 128 columns
@@ -285,7 +289,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             cur[32 + q] = __uint_as_float(v1[q]);
           }
         }
-        if (++buf == 2) { buf = 0; buf_phase ^= 1; }
+        if (++buf == NBUF) { buf = 0; buf_phase ^= 1; }
         if constexpr (LOG2 >= 1) {
           if ((i & 1) == 0) {
 #pragma unroll
@@ -295,7 +299,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           add_rn(cur, lvl0);
 #pragma unroll
           for (int lv = 1; lv < LOG2; lv++) {
-            const uint32_t slot = tmem + lane_off + (uint32_t)(2 * BN + (lv - 1) * BN) + col_off;
+            const uint32_t slot = tmem + lane_off + (uint32_t)(NBUF * BN + (lv - 1) * BN) + col_off;
             if (((i >> lv) & 1) == 0) {
               uint32_t w0[32], w1[32];
 #pragma unroll
@@ -374,7 +378,7 @@ static bi_status tree_partials_launch(const void *A, const void *W, float *out, 
   tree_schedule(p.leaves, p.merges);
   if (schedule_depth(p.leaves, p.merges) > STACK_SLOTS + 1) return BI_ERR_UNSUPPORTED_SHAPE;
   const int lps = p.leaves;
-  const bool wide = N % 128 == 0 && (lps == 1 || lps == 2 || lps == 4 || lps == 8);
+  const bool wide = N % 128 == 0 && (lps == 1 || lps == 2 || lps == 4 || lps == 8 || lps == 16);
   const int bn = wide ? 128 : 64;
   CUtensorMap tmA, tmW;
   if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
@@ -393,6 +397,7 @@ static bi_status tree_partials_launch(const void *A, const void *W, float *out, 
     case 2: ok = run(gemm_tree_kernel<128, 2>, Cfg<128>::SMEM); break;
     case 4: ok = run(gemm_tree_kernel<128, 4>, Cfg<128>::SMEM); break;
     case 8: ok = run(gemm_tree_kernel<128, 8>, Cfg<128>::SMEM); break;
+    case 16: ok = run(gemm_tree_kernel<128, 16>, Cfg<128>::SMEM); break;
     default: ok = run(gemm_tree_kernel<64, 0>, Cfg<64>::SMEM); break;
   }
   if (!ok) return BI_ERR_CUDA;

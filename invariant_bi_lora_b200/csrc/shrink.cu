@@ -149,6 +149,12 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   const int lr0 = mt * 16 + g, lr1 = lr0 + 8;       // local rows in the tile
   const bool v0 = lr0 < ti.rows, v1 = lr1 < ti.rows;
 
+  // token rows of this thread's fragment rows: their loads go out before
+  // the A staging, since the x loads wait on them
+  int row0 = 0, row1 = 0;
+  if (v0) row0 = tile_row(p.perm, ti, lr0);
+  if (v1) row1 = tile_row(p.perm, ti, lr1);
+
   // ---- shared memory holds the CTA's A slice (staged once, by every
   // thread with 16-byte cp.async, when it fits in 64 KB).  Rows are 128 bytes
   // per leaf; the 16-byte chunk index is XOR-ed with (row & 1) << 2 so that
@@ -175,9 +181,6 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   // global memory into a register ring of PF leaves; A fragments come from
   // the staged slice, or from global memory with the x ones when A is not
   // staged.
-  int row0 = 0, row1 = 0;
-  if (v0) row0 = tile_row(p.perm, ti, lr0);
-  if (v1) row1 = tile_row(p.perm, ti, lr1);
   const uint16_t *xr0 = p.x + (size_t)row0 * p.K + 8 * c;
   const uint16_t *xr1 = p.x + (size_t)row1 * p.K + 8 * c;
   const uint16_t *acol[NT];
