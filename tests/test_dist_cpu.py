@@ -1,4 +1,4 @@
-"""Multi-rank host logic on CPU process groups (gloo, world size 2).
+"""Multi-rank host logic on CPU process groups (gloo, world sizes 2 and 4).
 
 - max_over_ranks: the bench's device-time reduction (every rank gets the
   elementwise maximum).
@@ -88,9 +88,9 @@ def test_max_over_ranks_without_group():
     assert max_over_ranks([1, 2.5]) == [1.0, 2.5]
 
 
-def test_tp_tree_gemm_two_ranks(tmp_path):
+@pytest.mark.parametrize("world", [2, 4])
+def test_tp_tree_gemm_ranks(tmp_path, world):
     oracle.tree_sum(np.zeros(1, np.float32))        # build the oracle library before forking ranks
-    world = 2
     mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
     a, w = synth.gemm_inputs(M, N, K, seed=7)
