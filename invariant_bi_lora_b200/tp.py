@@ -55,13 +55,18 @@ def _gpu_combine(parts, out):
 def tree_gemm_tp(A_local: torch.Tensor, W_local: torch.Tensor, C: torch.Tensor,
                  group: Optional[dist.ProcessGroup] = None,
                  partial_fn: Optional[Callable] = None,
-                 combine_fn: Optional[Callable] = None) -> torch.Tensor:
+                 combine_fn: Optional[Callable] = None,
+                 check_finite: bool = False) -> torch.Tensor:
     """C = sum over ranks of A_q . W_q^T, reduced by the canonical tree.
 
     A_local [M][K/world] and W_local [N][K/world] (bf16, K-contiguous) are
     this rank's slices; C [M][N] fp32 receives the full result on every
     rank.  Collective: every rank of `group` must call it with the same M, N
-    and slice width."""
+    and slice width.  A rank that fails or leaves before the gather makes
+    the collective raise on the others (the process group's timeout bounds
+    the wait).  With check_finite, every rank inspects the gathered partials
+    before the combine and raises, naming the ranks, if any holds a NaN or an
+    infinity; all ranks see the same partials, so all raise together."""
     partial_fn = partial_fn or _gpu_partial
     combine_fn = combine_fn or _gpu_combine
     world = dist.get_world_size(group) if dist.is_initialized() else 1
@@ -77,6 +82,11 @@ def tree_gemm_tp(A_local: torch.Tensor, W_local: torch.Tensor, C: torch.Tensor,
     partial_fn(A_local, W_local, partial)
     parts = torch.empty(world * M, N, dtype=torch.float32, device=C.device)
     dist.all_gather_into_tensor(parts, partial, group=group)      # concatenated in rank order
+    if check_finite:
+        ok = torch.isfinite(parts.view(world, -1)).all(dim=1).tolist()
+        bad = [q for q, good in enumerate(ok) if not good]
+        if bad:
+            raise RuntimeError(f"tree_gemm_tp: non-finite partial from rank(s) {bad}")
     combine_fn(parts.view(world, M, N), C)
     return C
 

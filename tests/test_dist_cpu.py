@@ -10,6 +10,7 @@
   what is checked is the rank plumbing: K ranges, gather order, and that the
   result is the oracle's canonical tree over all leaves, bit for bit.
 """
+import datetime
 import os
 import socket
 
@@ -73,6 +74,59 @@ def _worker(rank, world, port, result_dir):
         np.save(os.path.join(result_dir, f"c{rank}.npy"), _bits(C))
     finally:
         dist.destroy_process_group()
+
+
+def _fault_worker(rank, world, port, result_dir, kind):
+    """Host-side failures: a rank whose partial is NaN (kind 'nan'), or a
+    rank that leaves before the collective (kind 'leave')."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    try:
+        if kind == "leave" and rank == world - 1:
+            return
+        a, w = synth.gemm_inputs(M, N, K, seed=3)
+        k0, k1 = shard_k_range(K, world, rank)
+        a_loc = torch.from_numpy(np.ascontiguousarray(a[:, k0:k1]).view(np.int16))
+        w_loc = torch.from_numpy(np.ascontiguousarray(w[:, k0:k1]).view(np.int16))
+
+        def partial_fn(A_local, W_local, out):
+            out.copy_(torch.from_numpy(oracle.tree_combine(
+                _leaf_values(A_local.numpy().view(np.uint16), W_local.numpy().view(np.uint16)))))
+            if kind == "nan" and rank == 1:
+                out[3, 5] = float("nan")
+
+        def combine_fn(parts, out):
+            out.copy_(torch.from_numpy(oracle.tree_combine(parts.numpy())))
+
+        C = torch.empty(M, N, dtype=torch.float32)
+        try:
+            tree_gemm_tp(a_loc, w_loc, C, partial_fn=partial_fn, combine_fn=combine_fn, check_finite=True)
+            msg = "no error"
+        except RuntimeError as e:
+            msg = str(e)
+        with open(os.path.join(result_dir, f"r{rank}.txt"), "w") as f:
+            f.write(msg)
+    finally:
+        if not (kind == "leave" and rank == world - 1):
+            try:
+                dist.destroy_process_group()
+            except Exception:
+                pass
+
+
+@pytest.mark.parametrize("kind", ["nan", "leave"])
+def test_tp_failures_are_reported(tmp_path, kind):
+    oracle.tree_sum(np.zeros(1, np.float32))
+    world = 2
+    mp.start_processes(_fault_worker, args=(world, _free_port(), str(tmp_path), kind), nprocs=world,
+                       join=True, start_method="spawn")
+    if kind == "nan":
+        for r in range(world):
+            assert "non-finite partial from rank(s) [1]" in (tmp_path / f"r{r}.txt").read_text(), r
+    else:
+        msg = (tmp_path / "r0.txt").read_text()
+        assert msg != "no error", msg           # the survivor's collective failed, it did not hang
 
 
 def test_shard_k_range():
