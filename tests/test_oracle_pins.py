@@ -392,6 +392,20 @@ def test_log_softmax_canon_lane_count(oracle_mod):
     assert f32bits(out[4097]) == f32bits(F32(F32(-17.0) - L))
 
 
+def test_log_softmax_canon_shift_invariance(oracle_mod):
+    """log_softmax(x + c) = log_softmax(x) exactly when every x - max is
+    exact in both: integer logits in [-40, 0] shifted by c = 2^20 (all
+    exactly representable, their differences exact).  This pins the order
+    of the output step: (x - max) - L; x - (max + L) would round max + L at
+    the scale of 2^20."""
+    g = np.random.default_rng(11)
+    x = g.integers(-40, 1, size=(3, 8192)).astype(np.float32)
+    a = oracle_mod.log_softmax_canon(x)
+    b = oracle_mod.log_softmax_canon(x + np.float32(2.0 ** 20))
+    assert np.array_equal(f32bits(a), f32bits(b))
+    assert not np.all(a == np.round(a))               # L is not an integer: the case is not trivial
+
+
 def test_log_softmax_canon_vs_exact(oracle_mod):
     x = synth.logits_inputs(4, 151936, seed=10)
     c = oracle_mod.log_softmax_canon(x).astype(np.float64)
