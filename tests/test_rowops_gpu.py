@@ -99,6 +99,14 @@ def test_log_softmax_wide_range_rows(R):
     assert np.array_equal(lsm(x), oracle.log_softmax_canon(x).view(np.uint32))
 
 
+def test_log_softmax_shift_invariance():
+    """Integer logits and the same logits + 2^20 give the same bits: every
+    x - max is exact in both, and the output is (x - max) - L."""
+    g = np.random.default_rng(11)
+    x = g.integers(-40, 1, size=(5, 151936)).astype(np.float32)
+    assert np.array_equal(lsm(x), lsm(x + np.float32(2.0 ** 20)))
+
+
 def test_exp_shortcut_matches_exp():
     """The log_softmax exp shortcut gives bi_exp's bits on [-87, 88]."""
     xs = np.concatenate([np.linspace(-87, 88, 1 << 20), -np.abs(np.random.default_rng(4).standard_normal(1 << 18) * 30)])
