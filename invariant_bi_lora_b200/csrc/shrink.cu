@@ -14,10 +14,11 @@
 //   leaves = combined by the canonical halving tree in fp32 (__fadd_rn).
 // A CTA owns a contiguous power-of-two block of leaves (one subtree).  Its
 // warps split that block into G contiguous groups (subtrees again); a warp
-// folds its group's leaves in post order on a register stack, the G group
-// values meet in shared memory (perfect tree), and in mode TREE the
-// `splits` CTAs of a row tile -- one thread-block cluster -- meet through
-// distributed shared memory, perfect tree again.  Every level is a level
+// folds its group's leaves in post order in registers, the G group values
+// meet in shared memory (perfect tree), and in mode TREE the `splits` CTAs
+// of a row tile -- one thread-block cluster -- meet through distributed
+// shared memory (a reduce-scatter of pushes, one cluster barrier), perfect
+// tree again.  Every level is a level
 // of the one canonical tree over the K/64 leaves, so the bits cannot depend
 // on how the work was cut.
 //
@@ -26,10 +27,11 @@
 // 128-bit load, for x and for A alike.  Inside a 32-wide k chunk, thread
 // (g, c) feeds k = 8c..8c+7 to MMA k-slots {2c, 2c+1, 2c+8, 2c+9} of two
 // MMAs; the same permutation is applied to both operands, so the products
-// summed are exactly x[m][k] * A[j][k].  No shared-memory staging: the loads
-// go straight to registers through a ring of PF leaves per warp, so every
-// warp keeps PF leaves of loads in flight while it multiplies -- the kernel
-// is HBM-bound, and the ring depth is what hides DRAM latency.
+// summed are exactly x[m][k] * A[j][k].  x is not staged in shared memory:
+// its loads go straight to registers through a ring of PF leaves per warp,
+// so every warp keeps PF leaves of loads in flight while it multiplies.  The
+// CTA's slice of A (read by all its warps) is staged once in shared memory
+// when it fits in 64 KB.
 #include "tc.cuh"
 
 #include <cooperative_groups.h>
