@@ -62,6 +62,7 @@ def _load():
         "or_shrink_exact": (None, [P, P, P, L, L, L, L, P, P, I]),
         "or_expand_exact": (None, [P, P, P, L, L, L, L, P, P, P, I]),
         "or_gemm_exact": (None, [P, P, L, L, L, P, L, P, P, I]),
+        "or_addmm_exact": (None, [P, P, P, L, L, L, P, L, P, P, I]),
         "or_segment": (None, [P, L, I, P, P]),
         "or_rmsnorm_exact": (None, [P, P, L, L, D, P, I]),
         "or_rmsnorm_canon": (None, [P, P, L, L, F, P, I]),
@@ -221,6 +222,27 @@ def gemm_exact(a, w, rows=None, nthreads=None):
     b = np.empty((nr, N), np.float64)
     _load().or_gemm_exact(_p(a), _p(w), M, N, K, rp, nr if rows is not None else 0,
                           _p(C), _p(b), _nt(nthreads))
+    return C, b
+
+
+def addmm_exact(bias, a, w, rows=None, nthreads=None):
+    """bias bf16 [N]; a bf16 [M,K]; w bf16 [N,K]; C = bias + a @ w.T in
+    fp64 (torch.addmm).  rows: optional index list.  Returns (C, bound)
+    with bound = |bias| + sum |a*w|."""
+    bias = _c(bias, np.uint16)
+    a = _c(a, np.uint16)
+    w = _c(w, np.uint16)
+    M, K = a.shape
+    N = w.shape[0]
+    assert w.shape == (N, K) and bias.shape == (N,)
+    rp, nr = None, M
+    if rows is not None:
+        rows = _c(rows, np.int64)
+        rp, nr = _p(rows), rows.size
+    C = np.empty((nr, N), np.float64)
+    b = np.empty((nr, N), np.float64)
+    _load().or_addmm_exact(_p(bias), _p(a), _p(w), M, N, K, rp, nr if rows is not None else 0,
+                           _p(C), _p(b), _nt(nthreads))
     return C, b
 
 

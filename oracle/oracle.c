@@ -308,6 +308,21 @@ void or_gemm_exact(const uint16_t *A, const uint16_t *W, long M, long N, long K,
     }
 }
 
+/* addmm ["Batch Invariant Ops", Highlighted Details: torch.addmm], exact:
+ *   C[m][n] = bias[n] + sum_k A[m][k] * W[n][k]
+ * bias bf16 [N]; the rest as or_gemm_exact.  bound = |bias| + sum |a*w|. */
+void or_addmm_exact(const uint16_t *bias, const uint16_t *A, const uint16_t *W, long M, long N, long K,
+                    const long *rows, long nrows, double *C, double *bound, int nthreads)
+{
+    or_gemm_exact(A, W, M, N, K, rows, nrows, C, bound, nthreads);
+    long R = rows ? nrows : M;
+    for (long i = 0; i < R; i++)
+        for (long n = 0; n < N; n++) {
+            C[i * N + n] += bf(bias[n]);
+            if (bound) bound[i * N + n] += fabs(bf(bias[n]));
+        }
+}
+
 /* Segment build: stable counting sort of token indices by adapter id.
  * offsets[a] = number of tokens with id < a (offsets[n_ad] = number of
  * tokens with a valid id); perm[offsets[a] + i] = the i-th token, in

@@ -5,13 +5,11 @@ test_oracle_pins.py fails.  The mutant is compiled into a temporary library
 and swapped into the oracle module for the duration of the test; the
 checked-in oracle is untouched.  CPU only.
 
-Not in the list, because no CPU pin can see them: changes that stay inside
+Not in the list, because no CPU pin can see it: a change that stays inside
 the accuracy bounds of the written exp/log (a coefficient of the log
-series changed from 1/9 to 1/8 moves its result by far less than an ulp),
-and reassociating RMSNorm's two final products (x*w*inv against
-x*inv*w), which differ by at most an ulp before the bf16 rounding.  Both
-would be caught by the GPU parity tests, which compare the kernels with
-the oracle bit for bit."""
+series changed from 1/9 to 1/8 moves its result by far less than an ulp).
+The GPU parity tests, which compare the kernels with the oracle bit for
+bit, would catch it."""
 import inspect
 
 import pytest
@@ -28,6 +26,8 @@ MUTANTS = [
     ("exp: ln2 tail dropped", "    r = fmaf(-n, ln2_tl, r);\n", "\n"),
     ("log: no reduction to [sqrt(1/2), sqrt(2))", "if (m > sqrt2) { m = m * 0.5f; e = e + 1; }", ""),
     ("rmsnorm: eps outside the sqrt", "return 1.0f / sqrtf(ms + eps);", "return 1.0f / (sqrtf(ms) + eps);"),
+    ("rmsnorm: final products reassociated", "float v = or_bf16_to_f32(xr[k]) * inv;\n            y[i * n + k] = or_f32_to_bf16(v * or_bf16_to_f32(w[k]));",
+     "float v = inv * or_bf16_to_f32(w[k]);\n            y[i * n + k] = or_f32_to_bf16(or_bf16_to_f32(xr[k]) * v);"),
     ("log_softmax: reassociated output", "for (long k = 0; k < n; k++) out[i * n + k] = (xr[k] - m) - L;",
      "for (long k = 0; k < n; k++) out[i * n + k] = xr[k] - (m + L);"),
     ("log_softmax: 1024 lanes", "float S = or_canon_sum(e, n, 4096, 4);", "float S = or_canon_sum(e, n, 1024, 4);"),
@@ -39,6 +39,7 @@ MUTANTS = [
     ("expand: y not rounded to bf16", "yb[j] = (double)or_bf16_to_f32(or_f32_to_bf16(y[m * r + j]));",
      "yb[j] = (double)y[m * r + j];"),
     ("gemm: W read transposed", "double p = av[k] * bf(wr[k]);", "double p = av[k] * bf(W[k * N + n]);"),
+    ("addmm: bias indexed by row", "C[i * N + n] += bf(bias[n]);", "C[i * N + n] += bf(bias[i % N]);"),
     ("segment: tokens scattered in reverse order",
      "if (ids[t] >= 0 && ids[t] < n_ad) perm[count[ids[t]]++] = (int32_t)t;",
      "if (ids[M - 1 - t] >= 0 && ids[M - 1 - t] < n_ad) perm[count[ids[M - 1 - t]]++] = (int32_t)(M - 1 - t);"),

@@ -272,6 +272,37 @@ def test_gemm_exact(oracle_mod):
     Cr, br = oracle_mod.gemm_exact(a, w, rows=rows)
     assert np.array_equal(Cr, C[rows]) and np.array_equal(br, b[rows])
 
+def test_addmm_exact_pins(oracle_mod):
+    """torch.addmm's value, exact: bias + a @ w.T.  Pinned by numpy float64,
+    integer brute force, and two special cases (zero bias reduces to the
+    GEMM; zero operands give the bias)."""
+    M, N, K = 7, 48, 192
+    a, w = synth.gemm_inputs(M, N, K, seed=11)
+    bias = synth.normal_bf16((N,), 1.0, seed=11, tag=9)
+    C, bound = oracle_mod.addmm_exact(bias, a, w)
+    af, wf, bf = (oracle_mod.bf16_to_f32(v).astype(np.float64) for v in (a, w, bias))
+    np.testing.assert_allclose(C, bf[None, :] + af @ wf.T, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(bound, np.abs(bf)[None, :] + np.abs(af) @ np.abs(wf).T, rtol=1e-13)
+    zero = np.zeros(N, np.uint16)
+    C0, _ = oracle_mod.addmm_exact(zero, a, w)
+    G, _ = oracle_mod.gemm_exact(a, w)
+    assert np.array_equal(C0, G)
+    Cz, _ = oracle_mod.addmm_exact(bias, np.zeros_like(a), w)
+    assert np.array_equal(Cz, np.tile(bf, (M, 1)))
+    ai = synth.integer_bf16((5, 64), -4, 4, seed=2, tag=1)
+    wi = synth.integer_bf16((16, 64), -4, 4, seed=2, tag=2)
+    bi_ = synth.integer_bf16((16,), -100, 100, seed=2, tag=3)
+    Ci, _ = oracle_mod.addmm_exact(bi_, ai, wi)
+    A_i = oracle_mod.bf16_to_f32(ai).astype(np.int64)
+    W_i = oracle_mod.bf16_to_f32(wi).astype(np.int64)
+    want = oracle_mod.bf16_to_f32(bi_).astype(np.int64)[None, :] + np.array(
+        [[sum(int(A_i[m, k]) * int(W_i[n, k]) for k in range(64)) for n in range(16)] for m in range(5)])
+    assert np.array_equal(Ci, want.astype(np.float64))
+    rows = np.array([6, 0, 3])
+    Cr, _ = oracle_mod.addmm_exact(bias, a, w, rows=rows)
+    assert np.array_equal(Cr, C[rows])
+
+
 
 # ---------------------------------------------------------------- RMSNorm
 
@@ -316,6 +347,42 @@ def test_rmsnorm_canon_sum_order(oracle_mod):
     ones = np.full(n, 0x3F80, np.uint16)
     want = F32(F32(1.0) / np.sqrt(F32(F32(1.0) + F32(1e-6)), dtype=np.float32))
     assert f32bits(oracle_mod.rmsnorm_inv_canon(ones, 1e-6)) == f32bits(want)
+
+
+def test_rmsnorm_canon_product_order(oracle_mod):
+    """Rows x = k/16 with integer |k| <= 63, n = 4096: every x^2 is a
+    multiple of 1/256 and the whole sum stays below 2^16, so every partial
+    sum is exact and S = sum(k^2)/256 in any order.  inv = fl(1/fl(sqrt(
+    fl(fl(S/n) + eps)))) is then a closed form, and the reading of the RMSNorm
+    output is y = bf16(fl(fl(x * inv) * w)).  On these 512 rows (seed 2)
+    some outputs change under either other order of the two products,
+    x * (inv * w) or (x * w) * inv, so the pin tells the orders apart."""
+    R, n = 512, 4096
+    g = np.random.default_rng(2)
+    k = g.integers(-63, 64, size=(R, n))
+    x = (k / 16.0).astype(np.float32)
+    xb = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle_mod.bf16_to_f32(xb), x)                  # x is exact in bf16
+    w = torch.from_numpy((g.standard_normal(n) * 0.1 + 1.0).astype(np.float32)).to(torch.bfloat16)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    wf = w.float().numpy()
+    m = (k.astype(np.int64) ** 2).sum(axis=1)
+    assert np.all(m < 2 ** 24)
+    S = (m / 256.0).astype(np.float32)
+    assert np.all(S.astype(np.float64) == m / 256.0)
+    eps = F32(1e-6)
+    inv = (F32(1.0) / np.sqrt((S / F32(n)).astype(np.float32) + eps).astype(np.float32)).astype(np.float32)
+    inv = inv[:, None]
+
+    def bf16(v):
+        return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+    want = bf16((x * inv).astype(np.float32) * wf)
+    other1 = bf16(x * (inv * wf).astype(np.float32))
+    other2 = bf16((x * wf).astype(np.float32) * inv)
+    assert np.sum(want != other1) > 0 and np.sum(want != other2) > 0     # the pin discriminates
+    got = oracle_mod.rmsnorm_canon(xb, wb, eps=1e-6)
+    assert np.array_equal(got, want)
 
 
 def test_rmsnorm_canon_vs_exact(oracle_mod):
