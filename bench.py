@@ -44,21 +44,44 @@ WORKLOAD = ("segmented multi-adapter LoRA shrink M=4096 tokens, 8 adapters, K=40
             "split-K 8 tree, inside one pass of the whole deterministic-reduction path")
 L2_FLUSH_BYTES = 256 << 20
 
-# shrink algorithmic bytes (segmented, r=16): x + A + y + plan(perm + offsets)
 M4, K4, R4, NAD = 4096, 4096, 16, 8
-SHRINK_BYTES = M4 * K4 * 2 + NAD * R4 * K4 * 2 + M4 * R4 * 4 + 4 * (M4 + NAD + 2)
+PLAN_TILES = (M4 + 63) // 64 + NAD + 1
+
+
+def shrink_bytes(M=M4, K=K4, r=R4, n_ad=NAD):
+    """Algorithmic bytes of one segmented shrink: x, every adapter's A, y,
+    and the plan's token ids and 16-byte tile headers."""
+    return M * K * 2 + n_ad * r * K * 2 + M * r * 4 + 4 * M + 16 * ((M + 63) // 64 + n_ad + 1)
+
+
+def expand_bytes(M=M4, N=4096, r=R4, n_ad=NAD):
+    """y, every adapter's B, the fp32 out write and the token ids."""
+    return M * r * 4 + n_ad * N * r * 2 + M * N * 4 + 4 * M
+
+
+SHRINK_BYTES = shrink_bytes()
+
+
+# Nominal B200 figures (datasheet): the targets are stated against these.
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
 
 
 def peaks():
+    """Roofline denominators.  Every kernel here is timed alone (its own
+    graph, L2 flushed before it), so the tensor peak is the burst figure.
+    The nominal datasheet figures are reported beside them."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    nominal = {"hbm_gbs_nominal": NOMINAL_HBM_GBS, "bf16_tflops_nominal": NOMINAL_BF16_TFLOPS}
     try:
         d = json.load(open(path))
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "source": "measured"}
+                "source": "measured (MEASURED_PEAKS.json: copy GB/s, cuBLAS bf16 burst TFLOP/s)", **nominal}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-                "source": "fallback"}
+                "source": "fallback (earlier measurement on this pool: 6.65 TB/s copy, 1.59 PFLOP/s burst)",
+                **nominal}
 
 
 # --------------------------------------------------------------------- clocks
@@ -171,7 +194,8 @@ class Workload:
         bi = self.bi
         lsm_bytes = 4096 * 151936 * 8
         k = [
-            ("plan", lambda: bi.lora_plan(self.ids, NAD, self.plan), 4 * M4 + 4 * (M4 + NAD + 2), 0, "hbm", 1),
+            ("plan", lambda: bi.lora_plan(self.ids, NAD, self.plan),
+             4 * M4 + 4 * (M4 + NAD + 2) + 4 * M4 + 16 * PLAN_TILES, 0, "hbm", 1),
             ("shrink_tree_s8", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y, 8, "tree"),
              SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
             ("shrink_atomic_s8", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y_at, 8, "atomic"),
@@ -179,7 +203,7 @@ class Workload:
             ("shrink_unsplit", lambda: bi.lora_shrink_segmented(self.x, self.A, self.plan, self.y_un, 1, "unsplit"),
              SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
             ("expand", lambda: bi.lora_expand_segmented(self.y, self.B, self.plan, self.out),
-             M4 * R4 * 4 + NAD * 4096 * R4 * 2 + M4 * 4096 * 4 + 4 * M4, 2 * M4 * 4096 * R4, "hbm", 1),
+             expand_bytes(), 2 * M4 * 4096 * R4, "hbm", 1),
             ("shrink16_tree_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "tree"),
              16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
             ("shrink16_atomic_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "atomic"),
@@ -225,10 +249,11 @@ class Workload:
 
 KERNEL_REPS = 10      # reps per kernel graph in the per-kernel timing block
 
-# DRAM bytes (read + write) of one launch, from an ncu capture of the same
-# kernel and workload (dram__bytes_read.sum + dram__bytes_write.sum; see
-# profiles/log_softmax_rows256_v151936.md for the command).  Only kernels
-# unchanged since their capture are listed.
+# DRAM bytes (read + write) of one launch, dram__bytes_read.sum +
+# dram__bytes_write.sum from an ncu capture of the same kernel on the same
+# workload, stored here because ncu does not run inside the bench.  Only
+# kernels whose code is unchanged since their capture are listed; the JSON
+# line says that the figure is a stored capture.
 MEASURED_TRAFFIC = {"log_softmax": 2489417216 + 2431791616}
 
 
@@ -333,6 +358,23 @@ def run_ours(args, rank, world, device):
                 tk = replay_ms(g)
                 f1 = replay_ms(g_flush)
                 per[name].append(max(tk - 0.5 * (f0 + f1), 1e-6) / R)
+
+        def time_kernel(fn):
+            """The same difference timing for one more kernel (ms, median of 5)."""
+            g = capture(reps(fn), cs)
+            t = []
+            for _ in range(5):
+                f0 = replay_ms(g_flush)
+                tk = replay_ms(g)
+                f1 = replay_ms(g_flush)
+                t.append(max(tk - 0.5 * (f0 + f1), 1e-6) / R)
+            del g
+            return statistics.median(t)
+
+        sweep = None
+        if not args.no_sweep:
+            del g_kern
+            sweep = Sweep(bi, synth, wl).run(time_kernel, pk)
         clk = clocks.stop()
     for k, v in per.items():
         sys.stderr.write(f"kernel {k}: {[round(t * 1e3, 2) for t in v]} us\n")
@@ -349,14 +391,9 @@ def run_ours(args, rank, world, device):
         ms = per[name]
         gbs = nbytes / (ms * 1e-3) / 1e9
         tfl = flops / (ms * 1e-3) / 1e12 if flops else None
-        if bound == "tensor":
-            ach, peak, unit = tfl, pk["bf16_tflops_sustained"], "TFLOP/s"
-        else:
-            ach, peak, unit = gbs, pk["hbm_gbs"], "GB/s"
         kern.append({"name": name, "us": round(ms * 1e3, 3), "bytes": nbytes, "flops": flops,
                      "gbs": round(gbs, 1), "tflops": None if tfl is None else round(tfl, 2),
-                     "bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
-                     "frac": round(ach / peak, 4), "launches": launches})
+                     **roof(bound, gbs, tfl, pk), "launches": launches})
     by = {k["name"]: k for k in kern}
     dom = max(kern, key=lambda k: k["us"])
     tree = by["shrink_tree_s8"]
@@ -379,15 +416,21 @@ def run_ours(args, rank, world, device):
                              "replays just before and after it, CUDA events, median of 5"},
         "roofline": {"kernel": dom["name"], "bound": dom["bound"], "achieved": dom["achieved"],
                      "peak": dom["peak"], "unit": dom["unit"], "frac": dom["frac"],
-                     "traffic": MEASURED_TRAFFIC.get(dom["name"]), "peak_source": pk["source"]},
+                     "traffic": MEASURED_TRAFFIC.get(dom["name"]),
+                     "traffic_source": ("stored ncu capture of this kernel and workload (code unchanged since)"
+                                        if dom["name"] in MEASURED_TRAFFIC else None),
+                     "peak_source": pk["source"], "peak_nominal": dom["peak_nominal"],
+                     "frac_nominal": dom["frac_nominal"]},
         "shrink_roofline": {"bound": "hbm", "achieved": tree["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                            "frac": tree["frac"], "bytes_per_launch": SHRINK_BYTES},
+                            "frac": tree["frac"], "peak_nominal": NOMINAL_HBM_GBS,
+                            "frac_nominal": tree["frac_nominal"], "bytes_per_launch": SHRINK_BYTES},
         "delta_vs_atomic_pct": round(100.0 * (tree["us"] / by["shrink_atomic_s8"]["us"] - 1.0), 2),
         "speedup_vs_unsplit_pct": round(100.0 * (by["shrink_unsplit"]["us"] / tree["us"] - 1.0), 2),
         "bi_gemm_tflops": None if gemm is None else gemm["tflops"],
         "atomic_variation": atomic_var,
         "shrink16_cold_stream": stream16,
         "kernels": kern,
+        "sweep": sweep,
         "kernel_sum_ms": round(sum(per.values()), 4),
         "gpu_launches": args.steps * sum(k["launches"] for k in kern),
         "device_status": status,
@@ -395,6 +438,99 @@ def run_ours(args, rank, world, device):
         "e2e": e2e,
     }
     return line
+
+
+class Sweep:
+    """The measurement rows of the configurations beside the step's (each
+    timed alone like the step's kernels, outside the timed step region):
+      d2  RMSNorm / log_softmax / mean on the first R of the 4096 rows,
+          R in {1, 7, 64, 513, 4096} (R <= 64 is latency: read the us);
+      d3  batch-invariant GEMM, K = 4096, N in {4096, 14336},
+          M in {1, 16, 64, 256, 1024, 4096} (HBM-bound for M <= 64);
+      d4  segmented shrink (tree / atomic s=8, unsplit) and expand at
+          r in {8, 16, 64}, M = 4096, 8 adapters;
+      d5  tree GEMM K = 16384, N = 4096, M in {1, 128, 2048},
+          s in {1, 2, 4, 8} emulated shards (with the combine)."""
+
+    def __init__(self, bi, synth, wl):
+        self.bi, self.rows = bi, []
+        self.cases = []
+        R_ALL = (1, 7, 64, 513, 4096)
+        for R in R_ALL:
+            n = 4096
+            self.add("d2", f"rmsnorm R={R}", {"rows": R, "n": n}, "hbm", R * n * 4 + n * 2, 0,
+                     lambda R=R: bi.rmsnorm(wl.xr[:R], wl.wr, wl.yr[:R], 1e-6))
+            self.add("d2", f"log_softmax R={R}", {"rows": R, "n": 151936}, "hbm", R * 151936 * 8, 0,
+                     lambda R=R: bi.log_softmax(wl.logits[:R], wl.lsm[:R]))
+            self.add("d2", f"mean R={R}", {"rows": R, "n": 151936}, "hbm", R * 151936 * 4 + R * 4, 0,
+                     lambda R=R: bi.mean(wl.logits[:R], wl.mean[:R]))
+        a, w = synth.gemm_inputs(4096, 14336, 4096, seed=3)
+        self.ga, self.gw = dev_bf16(a), dev_bf16(w)
+        self.gc = torch.empty(4096, 14336, dtype=torch.float32, device="cuda")
+        for N in (4096, 14336):
+            for M in (1, 16, 64, 256, 1024, 4096):
+                bound = "hbm" if M <= 64 else "tensor"
+                A_, W_ = self.ga[:M], self.gw[:N]
+                C_ = self.gc.view(-1)[:M * N].view(M, N)
+                self.add("d3", f"gemm M={M} N={N}", {"M": M, "N": N, "K": 4096}, bound,
+                         2 * M * 4096 + 2 * N * 4096 + 4 * M * N, 2 * M * N * 4096,
+                         lambda A_=A_, W_=W_, C_=C_: bi.gemm(A_, W_, C_))
+        for r in (8, 16, 64):
+            d = synth.lora_inputs(M4, K4, r, n_adapters=NAD, N=4096, seed=0)
+            X, A, B = dev_bf16(d["x"]), dev_bf16(d["at"]), dev_bf16(d["bt"])
+            plan = bi.lora_plan(torch.from_numpy(d["ids"]).cuda(), NAD)
+            y = torch.empty(M4, r, dtype=torch.float32, device="cuda")
+            bi.lora_shrink_segmented(X, A, plan, y, 8, "tree")
+            for mode, s in (("tree", 8), ("atomic", 8), ("unsplit", 1)):
+                self.add("d4", f"shrink {mode} s={s} r={r}", {"M": M4, "K": K4, "r": r, "adapters": NAD, "splits": s},
+                         "hbm", shrink_bytes(r=r), 2 * M4 * K4 * r,
+                         lambda X=X, A=A, plan=plan, y=y, mode=mode, s=s: bi.lora_shrink_segmented(X, A, plan, y, s, mode))
+            self.add("d4", f"expand r={r}", {"M": M4, "N": 4096, "r": r, "adapters": NAD}, "hbm",
+                     expand_bytes(r=r), 2 * M4 * 4096 * r,
+                     lambda y=y, B=B, plan=plan: bi.lora_expand_segmented(y, B, plan, wl.out))
+        a, w = synth.gemm_inputs(2048, 4096, 16384, seed=1)
+        self.ta, self.tw = dev_bf16(a), dev_bf16(w)
+        self.tc = torch.empty(2048, 4096, dtype=torch.float32, device="cuda")
+        self.tws = torch.empty(bi.gemm_tree_ws_bytes(2048, 4096, 8), dtype=torch.uint8, device="cuda")
+        for M in (1, 128, 2048):
+            for s in (1, 2, 4, 8):
+                bound = "tensor" if M >= 2048 else "hbm"
+                A_, C_ = self.ta[:M], self.tc[:M]
+                self.add("d5", f"tree_gemm M={M} s={s}", {"M": M, "N": 4096, "K": 16384, "shards": s}, bound,
+                         2 * M * 16384 + 2 * 4096 * 16384 + 4 * M * 4096, 2 * M * 4096 * 16384,
+                         lambda A_=A_, C_=C_, s=s: bi.gemm_tree(A_, self.tw, C_, s, self.tws))
+
+    def add(self, row, name, cfg, bound, nbytes, flops, fn):
+        self.cases.append((row, name, cfg, bound, nbytes, flops, fn))
+
+    def run(self, time_kernel, pk):
+        out = []
+        for (row, name, cfg, bound, nbytes, flops, fn) in self.cases:
+            try:
+                fn()
+                torch.cuda.synchronize()
+                ms = time_kernel(fn)
+            except Exception as e:                     # a shape the library rejects
+                out.append({"row": row, "name": name, "config": cfg, "error": str(e)})
+                continue
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            tfl = flops / (ms * 1e-3) / 1e12 if flops else None
+            out.append({"row": row, "name": name, "config": cfg, "us": round(ms * 1e3, 3),
+                        "gbs": round(gbs, 1), "tflops": None if tfl is None else round(tfl, 2),
+                        **roof(bound, gbs, tfl, pk)})
+        return out
+
+
+def roof(bound, gbs, tfl, pk):
+    """achieved / peak / frac of one kernel: tensor-bound kernels against the
+    burst bf16 figure, HBM-bound ones against the copy bandwidth; the same
+    against the nominal datasheet figures in frac_nominal."""
+    if bound == "tensor":
+        ach, peak, nom, unit = tfl, pk["bf16_tflops"], pk["bf16_tflops_nominal"], "TFLOP/s"
+    else:
+        ach, peak, nom, unit = gbs, pk["hbm_gbs"], pk["hbm_gbs_nominal"], "GB/s"
+    return {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit, "frac": round(ach / peak, 4),
+            "peak_nominal": nom, "frac_nominal": round(ach / nom, 4)}
 
 
 def atomic_variation(wl, bi, replays=100):
@@ -511,6 +647,58 @@ def oracle_shrink_rate(seconds=10.0):
     return SHRINK_BYTES * passes / el / 1e9, nt, passes, el
 
 
+def cpu_family_baselines(budget_s=12.0):
+    """The oracle on the host cores for the other kernel families, each on a
+    bounded sample of its configuration, in the GPU line's units:
+    canonical-fp32 and fp64 paths of the row ops, the fp64 GEMM on sampled
+    rows, the fp64 expand and the canonical tree combine.  About budget_s
+    seconds in all."""
+    import oracle
+    from invariant_bi_lora_b200 import synth
+    nt = oracle.max_threads()
+    out = []
+    per = budget_s / 9.0
+
+    def timed(name, fn, unit_amount, unit, sample):
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            fn()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= per:
+                break
+        out.append({"name": name, "value": round(unit_amount * n / el, 4), "unit": unit, "cores": nt,
+                    "kind": "oracle", "sample": f"{n} x {sample} in {el:.2f} s"})
+
+    xr, wr = synth.rmsnorm_inputs(1024, 4096, seed=0)
+    b = 1024 * 4096 * 4 + 4096 * 2
+    timed("rmsnorm canonical fp32", lambda: oracle.rmsnorm_canon(xr, wr, nthreads=nt), b / 1e9, "GB/s",
+          "1024 rows x 4096")
+    timed("rmsnorm fp64", lambda: oracle.rmsnorm_exact(xr, wr, nthreads=nt), b / 1e9, "GB/s", "1024 rows x 4096")
+    lg = synth.logits_inputs(64, 151936, seed=0)
+    timed("log_softmax canonical fp32", lambda: oracle.log_softmax_canon(lg, nthreads=nt),
+          64 * 151936 * 8 / 1e9, "GB/s", "64 rows x 151936")
+    timed("log_softmax fp64", lambda: oracle.log_softmax_exact(lg, nthreads=nt),
+          64 * 151936 * 8 / 1e9, "GB/s", "64 rows x 151936")
+    timed("mean canonical fp32", lambda: oracle.mean_canon(lg, nthreads=nt), 64 * 151936 * 4 / 1e9, "GB/s",
+          "64 rows x 151936")
+    timed("mean fp64", lambda: oracle.mean_exact(lg, nthreads=nt), 64 * 151936 * 4 / 1e9, "GB/s",
+          "64 rows x 151936")
+    a, w = synth.gemm_inputs(4096, 4096, 4096, seed=0)
+    rows = np.arange(0, 4096, 256)
+    timed("gemm fp64 (sampled rows)", lambda: oracle.gemm_exact(a, w, rows=rows, nthreads=nt),
+          2 * rows.size * 4096 * 4096 / 1e12, "TFLOP/s", f"{rows.size} of 4096 rows, N=K=4096")
+    d = synth.lora_inputs(512, 64, 16, n_adapters=NAD, N=4096, seed=0)
+    yv = np.random.default_rng(0).standard_normal((512, 16)).astype(np.float32)
+    timed("expand fp64", lambda: oracle.expand_exact(yv, d["bt"], d["ids"], nthreads=nt),
+          expand_bytes(M=512) / 1e9, "GB/s", "512 tokens, N=4096, r=16, 8 adapters")
+    parts = np.random.default_rng(1).standard_normal((8, 1 << 20)).astype(np.float32)
+    timed("tree combine canonical fp32", lambda: oracle.tree_combine(parts, nthreads=nt), 9 * 4 * (1 << 20) / 1e9,
+          "GB/s", "8 partials of 2^20")
+    return out
+
+
 def cpu_baseline_entry(seconds):
     v, nt, passes, el = oracle_shrink_rate(seconds)
     return {"value": round(v, 3), "unit": "GB/s", "cores": nt, "kind": "oracle",
@@ -542,6 +730,73 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------- one-op cases (ncu)
+
+CASES = ("plan", "shrink", "shrink_segmented", "expand_segmented", "gemm", "tree_gemm", "rmsnorm",
+         "log_softmax", "mean")
+CASE_DEFAULTS = {"M": 16384, "K": 4096, "N": 4096, "r": 16, "adapters": 8, "splits": 8, "mode": "tree",
+                 "shards": 8, "rows": 4096, "n": 151936}
+
+
+def run_case(a):
+    """One library operation on seeded inputs, --iters times back to back
+    (no timing): the command line of the ncu summaries.  Inputs are drawn
+    once and stay on the device."""
+    from invariant_bi_lora_b200 import bi, synth
+    torch.cuda.set_device(0)
+    op = a.case
+    if op in ("plan", "shrink", "shrink_segmented", "expand_segmented"):
+        d = synth.lora_inputs(a.M, a.K, a.r, n_adapters=a.adapters,
+                              N=a.N if op == "expand_segmented" else 0, seed=0)
+        X, A = dev_bf16(d["x"]), dev_bf16(d["at"])
+        y = torch.empty(a.M, a.r, dtype=torch.float32, device="cuda")
+        ids = torch.from_numpy(d["ids"]).cuda()
+        plan = bi.lora_plan(ids, a.adapters)
+        if op == "plan":
+            run = lambda: bi.lora_plan(ids, a.adapters, plan)
+        elif op == "shrink":
+            A0 = A[0].contiguous()
+            run = lambda: bi.lora_shrink(X, A0, y, a.splits, a.mode)
+        elif op == "shrink_segmented":
+            run = lambda: bi.lora_shrink_segmented(X, A, plan, y, a.splits, a.mode)
+        else:
+            B = dev_bf16(d["bt"])
+            out = torch.empty(a.M, a.N, dtype=torch.float32, device="cuda")
+            bi.lora_shrink_segmented(X, A, plan, y, a.splits, "tree")
+            run = lambda: bi.lora_expand_segmented(y, B, plan, out)
+    elif op in ("gemm", "tree_gemm"):
+        g_a, g_w = synth.gemm_inputs(a.M, a.N, a.K, seed=0)
+        GA, GW = dev_bf16(g_a), dev_bf16(g_w)
+        C = torch.empty(a.M, a.N, dtype=torch.float32, device="cuda")
+        if op == "gemm":
+            run = lambda: bi.gemm(GA, GW, C)
+        else:
+            ws = torch.empty(max(1, bi.gemm_tree_ws_bytes(a.M, a.N, a.shards)), dtype=torch.uint8, device="cuda")
+            run = lambda: bi.gemm_tree(GA, GW, C, a.shards, ws)
+    elif op == "rmsnorm":
+        x, w = synth.rmsnorm_inputs(a.rows, a.n, seed=0)
+        X, W = dev_bf16(x), dev_bf16(w)
+        Y = torch.empty_like(X)
+        run = lambda: bi.rmsnorm(X, W, Y)
+    elif op in ("log_softmax", "mean"):
+        X = torch.from_numpy(synth.logits_inputs(a.rows, a.n, seed=0)).cuda()
+        if op == "log_softmax":
+            O = torch.empty_like(X)
+            run = lambda: bi.log_softmax(X, O)
+        else:
+            O = torch.empty(a.rows, dtype=torch.float32, device="cuda")
+            run = lambda: bi.mean(X, O)
+    else:
+        raise SystemExit(f"unknown case {op}; one of {', '.join(CASES)}")
+    for _ in range(a.iters):
+        run()
+    torch.cuda.synchronize()
+    st = bi.get_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st}")
+    print(f"{op}: {a.iters} runs ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -551,6 +806,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--eager-only", action="store_true",
                     help="launch the step's kernels eagerly and exit (for ncu launch lists)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-configuration measurement rows (d2-d5)")
+    ap.add_argument("--case", default=None,
+                    help="run one library operation on seeded inputs --iters times and exit "
+                         "(for profiler captures): " + ", ".join(CASES))
+    ap.add_argument("--iters", type=int, default=3)
+    for k, v in CASE_DEFAULTS.items():
+        ap.add_argument(f"--{k}", type=type(v), default=v)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -559,14 +822,21 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.case:
+        run_case(args)
+        return
+
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
 
-    # CPU baseline first (rank 0, N=1 only), before any GPU work.
-    cpu = cpu_baseline_entry(args.cpu_seconds) if (rank == 0 and world == 1 and not args.eager_only) else None
+    # CPU baselines first (rank 0, N=1 only), before any GPU work.
+    cpu, cpu_families = None, None
+    if rank == 0 and world == 1 and not args.eager_only:
+        cpu = cpu_baseline_entry(args.cpu_seconds)
+        cpu_families = cpu_family_baselines(min(12.0, 1.2 * args.cpu_seconds))
 
     torch.cuda.set_device(local)
     if world > 1:
@@ -580,6 +850,7 @@ def main():
             torch.distributed.destroy_process_group()
     if rank == 0:
         line["cpu_baseline"] = cpu
+        line["cpu_baselines_other"] = cpu_families
         print(json.dumps(line), flush=True)
 
 

@@ -103,7 +103,13 @@ bi_status bi_lora_shrink(const void *x, const void *A, float *y,
 /*   Plan layout (int32): perm[M] (token indices, grouped by adapter,   */
 /*   increasing within a group), then offsets[n_adapters + 2] where     */
 /*   segment a is perm[offsets[a] .. offsets[a+1]), a = n_adapters being */
-/*   the "no adapter" segment.  1 <= n_adapters <= 256.                 */
+/*   the "no adapter" segment; then zero padding up to a multiple of 4  */
+/*   words, then a tile table of ceil(M/64) + n_adapters + 1 records of */
+/*   68 words, one per 64-row tile of the segments in order: {adapter,  */
+/*   rows (1..64), first perm position, 0, token ids[64] (-1 past      */
+/*   rows)}; records past the last tile have adapter -1.  The segmented */
+/*   kernels read their tile's adapter and rows from one record.       */
+/*   1 <= n_adapters <= 256.                                            */
 /* ------------------------------------------------------------------ */
 size_t bi_lora_plan_bytes(int M, int n_adapters);
 bi_status bi_lora_plan(const int32_t *ids, int M, int n_adapters,
@@ -124,8 +130,9 @@ bi_status bi_lora_shrink_segmented(const void *x, const void *A, const void *pla
  * or a latency-critical loop where an allocation (which may synchronise the
  * device) is not acceptable.  This call takes the adapter ids (int32 [M],
  * device) instead of a plan and builds the plan in a fixed array of the
- * library's own device memory: BI_NOALLOC_MAX_TOKENS + 258 int32 (about
- * 257 KiB), held by every GPU that loads the library until the process exits.
+ * library's own device memory, sized for BI_NOALLOC_MAX_TOKENS tokens and
+ * 256 adapters (152,904 int32, about 598 KiB), held by every GPU that loads
+ * the library until the process exits.
  * It allocates nothing.  Other arguments, results and guarantees are those of
  * bi_lora_plan followed by bi_lora_shrink_segmented (same bits).
  * M > BI_NOALLOC_MAX_TOKENS or n_adapters > 256 returns
@@ -162,13 +169,25 @@ bi_status bi_lora_expand_segmented(const float *y, const void *B, const void *pl
 /*   C[m][n] = sum_k A[m][k] * W[n][k]                                  */
 /* A bf16 [M][K], W bf16 [N][K]; C fp32 [M][N] (c_bf16 = 0) or bf16     */
 /* (c_bf16 = 1, round to nearest even from the fp32 accumulator).       */
-/* One locked tcgen05 configuration (128 x 256 tiles, K stepped 0 -> K  */
-/* in 64-wide stages, never split) whatever M is, so row m of C is      */
-/* bitwise the same for every M.  Requirements: K % 64 == 0, N % 16 ==  */
-/* 0, A / W / C 16-byte aligned.                                        */
+/* One locked tcgen05 reduction order (K stepped 0 -> K in 64-wide     */
+/* stages, one fp32 TMEM accumulator per element, never split) whatever */
+/* M is, so row m of C is bitwise the same for every M.  The output     */
+/* tile is 128 x 256, or 128 x 64 / 128 x 32 when M <= 512 / M <= 128 so */
+/* that small batches still spread the weight read; the accumulation of */
+/* an element does not depend on the tile width.  Requirements: K % 64  */
+/* == 0, N % 16 == 0, A / W / C 16-byte aligned.                        */
 /* ------------------------------------------------------------------ */
 bi_status bi_gemm(const void *A, const void *W, void *C, int M, int N, int K,
                   int c_bf16, bi_stream_t stream);
+
+/* Batch-invariant addmm ["Batch Invariant Ops", Highlighted Details:     */
+/* torch.addmm]:  C[m][n] = fl(acc[m][n] + bias[n]), acc being bi_gemm's */
+/* fp32 accumulator (same tiles, same K order), so C is bitwise bi_gemm's */
+/* fp32 result plus the bias in one IEEE fp32 addition, then the optional */
+/* bf16 rounding (c_bf16 = 1).  bias bf16 [N] (device, 16-byte aligned); */
+/* everything else as bi_gemm.                                           */
+bi_status bi_addmm(const void *bias, const void *A, const void *W, void *C, int M, int N, int K,
+                   int c_bf16, bi_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* TP-invariant tree GEMM [TBIK Abstract]: C = A . W^T with K cut into  */

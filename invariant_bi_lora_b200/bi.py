@@ -42,6 +42,7 @@ _SIGS = {
     "bi_lora_expand": (I, [P, P, P, I, I, I, I, P]),
     "bi_lora_expand_segmented": (I, [P, P, P, I, P, I, I, I, I, P]),
     "bi_gemm": (I, [P, P, P, I, I, I, I, P]),
+    "bi_addmm": (I, [P, P, P, P, I, I, I, I, P]),
     "bi_gemm_tree_ws_bytes": (Z, [I, I, I]),
     "bi_gemm_tree_partials": (I, [P, P, P, I, I, I, I, P]),
     "bi_gemm_tree": (I, [P, P, P, I, I, I, I, P, Z, P]),
@@ -216,6 +217,23 @@ def gemm(A, W, C, stream=None):
     if W.shape[1] != K or tuple(C.shape) != (M, N):
         raise ValueError("shape mismatch")
     _call("bi_gemm", _ptr(A), _ptr(W), _ptr(C), M, N, K, int(C.dtype == torch.bfloat16), _stream(stream))
+    return C
+
+
+def addmm(bias, A, W, C, stream=None):
+    """C[M,N] = bias[N] + A[M,K] . W[N,K]^T (torch.addmm); bias bf16, C fp32 or bf16."""
+    _check(bias, "bias", torch.bfloat16, 1)
+    _check(A, "A", torch.bfloat16, 2)
+    _check(W, "W", torch.bfloat16, 2)
+    if C.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("C must be float32 or bfloat16")
+    _check(C, "C", C.dtype, 2)
+    M, K = A.shape
+    N = W.shape[0]
+    if W.shape[1] != K or tuple(C.shape) != (M, N) or bias.shape[0] != N:
+        raise ValueError("shape mismatch")
+    _call("bi_addmm", _ptr(bias), _ptr(A), _ptr(W), _ptr(C), M, N, K, int(C.dtype == torch.bfloat16),
+          _stream(stream))
     return C
 
 

@@ -118,7 +118,7 @@ bi_status tree_combine_launch(const float *partials, float *out, int s, size_t c
   p.s = s;
   tree_schedule(s, p.merges);
   const size_t nv = count / 4;
-  const unsigned blocks = (unsigned)std::min<size_t>((nv + 255) / 256, 148 * 8);
+  const unsigned blocks = (unsigned)std::min<size_t>((nv + 255) / 256, (size_t)num_sms() * 8);
   switch (s) {
     case 2: tree_combine_pow2_kernel<2><<<blocks, 256, 0, stream>>>(partials, out, nv); break;
     case 4: tree_combine_pow2_kernel<4><<<blocks, 256, 0, stream>>>(partials, out, nv); break;

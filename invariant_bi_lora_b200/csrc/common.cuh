@@ -27,6 +27,8 @@ BI_DEV void flag_error(unsigned *status, unsigned code) {
 
 // Host side: address of the status word on the current device.
 unsigned *status_word();
+// Host side: SM count of the current device.
+int num_sms();
 
 // ----------------------------------------------------------------------
 // bf16 <-> fp32.  A bf16 value is the top half of an fp32 value, so the
@@ -58,10 +60,12 @@ BI_DEV uint4 ldg128_stream(const void *p) {
 // ----------------------------------------------------------------------
 // Warp-level mma.sync m16n8k16, bf16 inputs, fp32 accumulate:
 //   d = a . b + c
+// Not volatile: the compiler may move it past other instructions (it has no
+// effect beyond its outputs), so independent chains can be interleaved.
 // ----------------------------------------------------------------------
 BI_DEV void mma_bf16_16816(float d[4], const uint32_t a[4], const uint32_t b[2],
                            const float c[4]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
@@ -143,6 +147,27 @@ BI_DEV void resolve_tile_block(const int32_t *offsets, int n_ad, int M, int tile
 // Token index of position `pos` of a tile (identity without a plan).
 BI_DEV int tile_row(const int32_t *perm, const TileInfo &ti, int local) {
   return perm ? perm[ti.seg_begin + ti.row0 + local] : ti.row0 + local;
+}
+
+// ----------------------------------------------------------------------
+// Plan layout (int32 words), written by bi_lora_plan:
+//   perm[M]                 token indices grouped by adapter
+//   offsets[n_ad + 2]       segment starts in perm
+//   (zero to three words of padding: the table starts on 16 bytes)
+//   table[plan_tiles(M, n_ad)][kPlanRec]
+// Table record i describes the i-th 64-row tile of the segments taken in
+// order (segment a's tiles are its positions offsets[a] + 64j ...):
+//   {adapter (n_ad = no adapter, -1 = past the last tile), rows (1..64),
+//    first perm position, 0, token ids[64]} -- ids past `rows` are -1.
+// A kernel finds its tile's adapter and every token row in one read of
+// 272 bytes, instead of reading the offsets, then perm, then x.
+// ----------------------------------------------------------------------
+constexpr int kPlanTile = 64;
+constexpr int kPlanRec = 4 + kPlanTile;
+__host__ __device__ constexpr long plan_table_word(long M, int n_ad) { return (M + n_ad + 2 + 3) & ~3L; }
+__host__ __device__ constexpr long plan_tiles(long M, int n_ad) { return (M + kPlanTile - 1) / kPlanTile + n_ad + 1; }
+__host__ __device__ constexpr long plan_words(long M, int n_ad) {
+  return plan_table_word(M, n_ad) + kPlanRec * plan_tiles(M, n_ad);
 }
 
 }  // namespace bi

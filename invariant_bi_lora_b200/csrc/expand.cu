@@ -184,7 +184,7 @@ extern "C" bi_status bi_lora_expand_segmented(const float *y, const void *B, con
                                               int n_adapters, float *out, int M, int r, int N,
                                               int accumulate, bi_stream_t stream) {
   if (M > 0 && !plan) return BI_ERR_INVALID_ARG;
-  if (n_adapters < 1 || n_adapters > 256) return BI_ERR_INVALID_ARG;
+  if (n_adapters < 1 || n_adapters > bi::kMaxAdapters) return BI_ERR_INVALID_ARG;
   const int32_t *perm = static_cast<const int32_t *>(plan);
   return bi::expand_launch(y, B, perm, perm + M, n_adapters, out, M, r, N, accumulate,
                            reinterpret_cast<cudaStream_t>(stream));

@@ -7,20 +7,27 @@
 // with one consistent reduction order.  "Batch Invariant Ops" (Highlighted
 // Details): torch.mm.
 //
-// Locked policy: every call, whatever M is, uses the same 128 x 256 output
-// tile, steps K from 0 to K in 64-wide stages, accumulates each output
-// element in one TMEM accumulator by tcgen05.mma (M=128, N=256, K=16, bf16
-// in, fp32 accumulate) and never splits K.  Row m of C is therefore the
-// same bits for every M; rows past M are zero-filled by TMA and dropped.
+// Locked policy: every call, whatever M is, steps K from 0 to K in 64-wide
+// stages and accumulates each output element in one TMEM accumulator by
+// tcgen05.mma (M=128, K=16, bf16 in, fp32 accumulate), never splitting K.
+// The accumulation of one output element is the same whatever the MMA's N
+// (tests compare N = 32, 64 and 256 bit for bit), so the output tile's
+// width is free: 128 x 256 tiles from M = 513 on, and narrower 128 x 64 or
+// 128 x 32 tiles below, so that a small-M call still spreads its weight read
+// over the SMs (N = 4096: 128 or 256 CTAs instead of 16).  Row m of C is
+// therefore the same bits for every M; rows past M are zero-filled by TMA
+// and dropped.  addmm adds a bf16 bias to the fp32 accumulator after the
+// last K stage: C = fl(acc + bias[n]), then the optional bf16 rounding.
 //
 // Pipeline (persistent, one CTA per SM, 192 threads):
-//   warp 0      TMA producer: A and W tiles into a 4-stage shared ring
-//               (128-byte swizzle; 48 KB a stage)
+//   warp 0      TMA producer: A and W tiles into a shared ring
+//               (128-byte swizzle; 4 x 48 KB for 256-wide tiles, 8 stages
+//               for the narrow ones)
 //   warp 1      TMEM allocator and MMA issuer (one elected thread)
 //   warps 2..5  epilogue: TMEM -> registers -> global (fp32 or bf16),
 //               lane quadrant = warp % 4
-// Two 256-column TMEM accumulators let the epilogue of tile i overlap the
-// MMAs of tile i+1.  Every wait is bounded (tc.cuh).
+// Two TMEM accumulators let the epilogue of tile i overlap the MMAs of
+// tile i+1.  Every wait is bounded (tc.cuh).
 #include "tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -29,33 +36,43 @@
 namespace bi {
 
 namespace gemm {
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;        // 48 KB
+constexpr int BM = 128, BK = 64;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;                   // 2 accumulators x 256
-constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
+// Per output-tile width BN: the W stage, the ring depth, TMEM columns.
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN >= 256 ? 4 : 8;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;   // two accumulators
+  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+};
 }  // namespace gemm
 
+template <int STAGES>
 struct GemmSmemTail {
-  uint64_t full[gemm::STAGES];
-  uint64_t empty[gemm::STAGES];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint32_t tmem_base;
   uint32_t bail;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                 void *__restrict__ C, int M, int N, int K, int c_bf16, unsigned *status) {
+                 void *__restrict__ C, const uint16_t *__restrict__ bias, int M, int N, int K, int c_bf16,
+                 unsigned *status) {
   using namespace gemm;
+  constexpr int STAGES = Cfg<BN>::STAGES, B_BYTES = Cfg<BN>::B_BYTES, STAGE_BYTES = Cfg<BN>::STAGE_BYTES;
+  constexpr uint32_t TMEM_COLS = Cfg<BN>::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sa = smem;                                 // [STAGES][A_BYTES]
   uint8_t *sb = smem + STAGES * A_BYTES;              // [STAGES][B_BYTES]
-  GemmSmemTail *tail = reinterpret_cast<GemmSmemTail *>(smem + STAGES * STAGE_BYTES);
+  GemmSmemTail<STAGES> *tail = reinterpret_cast<GemmSmemTail<STAGES> *>(smem + STAGES * STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
@@ -164,6 +181,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_ld32(tbase + 32 * ch, v);
         tmem_wait_ld();
         const int col0 = nb * BN + 32 * ch;
+        if (bias && row < M) {
+          // addmm: one rounding, after the whole K reduction
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            const uint4 b = col0 + 8 * j < N ? __ldg(reinterpret_cast<const uint4 *>(bias + col0 + 8 * j))
+                                             : make_uint4(0, 0, 0, 0);
+            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+              v[8 * j + 2 * e] = __float_as_uint(__fadd_rn(__uint_as_float(v[8 * j + 2 * e]), bf16lo(bw[e])));
+              v[8 * j + 2 * e + 1] = __float_as_uint(__fadd_rn(__uint_as_float(v[8 * j + 2 * e + 1]), bf16hi(bw[e])));
+            }
+          }
+        }
         if (row < M) {
           if (!c_bf16) {
             float *dst = static_cast<float *>(C) + (size_t)row * N + col0;
@@ -239,32 +270,50 @@ int num_sms() {
   return cache[dev];
 }
 
-bi_status gemm_launch(const void *A, const void *W, void *C, int M, int N, int K, int c_bf16,
+template <int BN>
+static bi_status gemm_run(const void *A, const void *W, void *C, const void *bias, int M, int N, int K, int c_bf16,
+                          cudaStream_t stream) {
+  using namespace gemm;
+  CUtensorMap tmA, tmW;
+  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
+  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
+  constexpr size_t SMEM = Cfg<BN>::SMEM;
+  // per launch: the attribute belongs to the current device, and a process
+  // may drive several
+  if (cudaFuncSetAttribute(gemm_bf16_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) !=
+      cudaSuccess)
+    return BI_ERR_CUDA;
+  const long tiles = (long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)std::min<long>(tiles, num_sms());
+  gemm_bf16_kernel<BN><<<grid, THREADS, SMEM, stream>>>(tmA, tmW, C, static_cast<const uint16_t *>(bias), M, N, K,
+                                                       c_bf16 ? 1 : 0, status_word());
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status gemm_launch(const void *A, const void *W, void *C, const void *bias, int M, int N, int K, int c_bf16,
                       cudaStream_t stream) {
   using namespace gemm;
   if (M < 0 || N <= 0 || K <= 0) return BI_ERR_INVALID_ARG;
   if (M > 0 && (!A || !W || !C)) return BI_ERR_INVALID_ARG;
   if (K % BK != 0 || N % 16 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
-  if (!bi_aligned16(A) || !bi_aligned16(W) || !bi_aligned16(C)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (!bi_aligned16(A) || !bi_aligned16(W) || !bi_aligned16(C) || !bi_aligned16(bias)) return BI_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return BI_OK;
-  CUtensorMap tmA, tmW;
-  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
-  if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) != cudaSuccess)
-      return BI_ERR_CUDA;
-    attr_set = true;
-  }
-  const long tiles = (long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = (int)std::min<long>(tiles, num_sms());
-  gemm_bf16_kernel<<<grid, THREADS, SMEM, stream>>>(tmA, tmW, C, M, N, K, c_bf16 ? 1 : 0, status_word());
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  // the tile width only spreads the work (bit-neutral): narrow tiles when
+  // few rows would leave most SMs idle
+  if (M <= 128 && N % 32 == 0) return gemm_run<32>(A, W, C, bias, M, N, K, c_bf16, stream);
+  if (M <= 512 && N % 64 == 0) return gemm_run<64>(A, W, C, bias, M, N, K, c_bf16, stream);
+  return gemm_run<256>(A, W, C, bias, M, N, K, c_bf16, stream);
 }
 
 }  // namespace bi
 
 extern "C" bi_status bi_gemm(const void *A, const void *W, void *C, int M, int N, int K, int c_bf16,
                              bi_stream_t stream) {
-  return bi::gemm_launch(A, W, C, M, N, K, c_bf16, reinterpret_cast<cudaStream_t>(stream));
+  return bi::gemm_launch(A, W, C, nullptr, M, N, K, c_bf16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_addmm(const void *bias, const void *A, const void *W, void *C, int M, int N, int K,
+                              int c_bf16, bi_stream_t stream) {
+  if (M > 0 && !bias) return BI_ERR_INVALID_ARG;
+  return bi::gemm_launch(A, W, C, bias, M, N, K, c_bf16, reinterpret_cast<cudaStream_t>(stream));
 }

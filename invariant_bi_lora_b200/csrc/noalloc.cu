@@ -9,9 +9,9 @@
 // the adapter ids directly and keeps the plan in a fixed array of this
 // library's own device memory instead.
 //
-// The scratch is a file-scope __device__ array of kNoAllocMaxTokens + 258
-// int32 (about 257 KiB); every GPU that loads the library holds it until the
-// process exits.  Host code cannot use the array's name as a device address
+// The scratch is a file-scope __device__ array that holds the largest plan
+// (BI_NOALLOC_MAX_TOKENS tokens, 256 adapters: 152,904 int32, about 598 KiB);
+// every GPU that loads the library holds it until the process exits.  Host code cannot use the array's name as a device address
 // (on the host it names a stand-in object), so the first call on each device
 // looks the address up with cudaGetSymbolAddress, with that device current,
 // and caches it; that first call should therefore come before any stream
@@ -26,10 +26,11 @@
 namespace bi {
 
 constexpr int kNoAllocMaxTokens = BI_NOALLOC_MAX_TOKENS;
-constexpr int kNoAllocMaxAdapters = 256;
+constexpr int kNoAllocMaxAdapters = kMaxAdapters;
 
-// perm[M] followed by offsets[n_adapters + 2], as laid out by bi_lora_plan.
-static __device__ __align__(256) int32_t g_noalloc_plan[kNoAllocMaxTokens + kNoAllocMaxAdapters + 2];
+// A plan as bi_lora_plan lays it out (perm, offsets, tile table), at the
+// largest size this entry point accepts.
+static __device__ __align__(256) int32_t g_noalloc_plan[plan_words(kNoAllocMaxTokens, kNoAllocMaxAdapters)];
 
 static std::mutex g_noalloc_mu;
 static int32_t *g_noalloc_ptr[64];
@@ -61,7 +62,7 @@ extern "C" bi_status bi_lora_shrink_segmented_noalloc(const void *x, const void 
   int32_t *plan = nullptr;
   bi_status st = bi::noalloc_scratch(&plan);
   if (st != BI_OK) return st;
-  const size_t plan_bytes = sizeof(int32_t) * ((size_t)M + n_adapters + 2);
+  const size_t plan_bytes = sizeof(int32_t) * (size_t)bi::plan_words(M, n_adapters);
   st = bi_lora_plan(ids, M, n_adapters, plan, plan_bytes, stream);
   if (st != BI_OK) return st;
   return bi_lora_shrink_segmented(x, A, plan, n_adapters, y, M, K, r, splits, mode, stream);

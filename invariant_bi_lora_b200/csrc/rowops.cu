@@ -413,7 +413,7 @@ extern "C" bi_status bi_log_softmax(const float *x, float *out, int rows, int n,
 extern "C" bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream) {
   if ((n > 0 && (!x || !y)) || which < 0 || which > 3) return BI_ERR_INVALID_ARG;
   if (n == 0) return BI_OK;
-  const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 148 * 16);
+  const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, (size_t)bi::num_sms() * 16);
   bi::math_spec_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, which);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

@@ -27,11 +27,18 @@
 // 128-bit load, for x and for A alike.  Inside a 32-wide k chunk, thread
 // (g, c) feeds k = 8c..8c+7 to MMA k-slots {2c, 2c+1, 2c+8, 2c+9} of two
 // MMAs; the same permutation is applied to both operands, so the products
-// summed are exactly x[m][k] * A[j][k].  x is not staged in shared memory:
-// its loads go straight to registers through a ring of PF leaves per warp,
-// so every warp keeps PF leaves of loads in flight while it multiplies.  The
-// CTA's slice of A (read by all its warps) is staged once in shared memory
-// when it fits in 64 KB.
+// summed are exactly x[m][k] * A[j][k].  A CTA learns its tile (adapter and
+// token rows) from one read of the plan's tile table.  Two kernels, same
+// leaves and same tree, chosen by the grid size:
+//   ring: x goes straight to registers through a ring of PF leaves per
+//         warp, so every warp keeps PF leaves of loads in flight while it
+//         multiplies; the CTA's slice of A is staged once in shared memory
+//         when it fits in 64 KB.  Used when the grid needs more than one wave.
+//   bulk: the CTA's whole x and A slices are requested at once by the copy
+//         engine (one contiguous copy per row) into shared memory.  Used
+//         when every CTA of the grid is resident at once.
+// Each warp issues the MMAs of several leaves step by step across all of
+// their chains, so no MMA waits right behind the one it depends on.
 #include "tc.cuh"
 
 #include <cooperative_groups.h>
@@ -66,6 +73,11 @@ struct ShrinkParams {
   int a_offset;             // bytes from the start of dynamic shared memory to the A slice
   int g_offset;             // bytes to the exchange slots (mode TREE)
   int gather0;              // mode TREE: 1 = all partials to rank 0, 0 = reduce-scatter over the ranks
+  // bulk-copy kernel only
+  const int32_t *table;     // plan tile table (nullptr: rows in index order, adapter 0)
+  int sub;                  // CTA tiles per 64-row table record (64 / bm)
+  int rowbytes;             // bytes of one row's K range in one split (lc * 128)
+  int x_off, part_off;      // shared-memory offsets of the x rows and the group values
   uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
 };
 
@@ -77,26 +89,198 @@ struct LeafFrag {
   uint4 ab[2][NT];    // [chunk][n-tile]
 };
 
+// NL leaves at once: each leaf's value is, per n-tile, one chain of four
+// MMAs from zero -- k chunk 0 step 0, chunk 0 step 1, chunk 1 step 0,
+// chunk 1 step 1, always in that order.  The chains of different n-tiles
+// and leaves are independent, so they are issued step by step across all
+// of them: a chain's next MMA never waits right behind its previous one.
+template <int NT, int NL>
+BI_DEV void mma_leaves(float (&acc)[NL][NT][4], const LeafFrag<NT> (&f)[NL]) {
+#pragma unroll
+  for (int l = 0; l < NL; l++)
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int q = 0; q < 4; q++) acc[l][t][q] = 0.0f;
+#pragma unroll
+  for (int h = 0; h < 2; h++)
+#pragma unroll
+    for (int s = 0; s < 2; s++)
+#pragma unroll
+      for (int l = 0; l < NL; l++) {
+        const uint4 r0 = f[l].xa[h][0], r1 = f[l].xa[h][1];
+        const uint32_t a[4] = {s ? r0.z : r0.x, s ? r1.z : r1.x, s ? r0.w : r0.y, s ? r1.w : r1.y};
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+          const uint4 b = f[l].ab[h][t];
+          const uint32_t bb[2] = {s ? b.z : b.x, s ? b.w : b.y};
+          mma_bf16_16816(acc[l][t], a, bb, acc[l][t]);
+        }
+      }
+}
+
 // One leaf: four MMAs per n-tile (two k chunks x two k16 steps), from zero.
 template <int NT>
 BI_DEV void mma_leaf(float acc[NT][4], const LeafFrag<NT> &f) {
+  float a1[1][NT][4];
+  const LeafFrag<NT> f1[1] = {f};
+  mma_leaves<NT, 1>(a1, f1);
 #pragma unroll
   for (int t = 0; t < NT; t++)
 #pragma unroll
-    for (int q = 0; q < 4; q++) acc[t][q] = 0.0f;
+    for (int q = 0; q < 4; q++) acc[t][q] = a1[0][t][q];
+}
+
+// Binary-counter fold of leaf i (an index known at compile time) into the
+// pending subtree values lv: leaf i closes the levels where its index has a
+// 1 bit (left = the parked subtree, right = the one just finished) and parks
+// the result at its lowest 0 bit.  After the last leaf of a power-of-two
+// group, acc holds the group's subtree value.
+template <int NT, int LOG2>
+BI_DEV void fold_leaf(int i, float (&lv)[LOG2 > 0 ? LOG2 : 1][NT][4], float (&acc)[NT][4]) {
 #pragma unroll
-  for (int h = 0; h < 2; h++) {
-    const uint4 r0 = f.xa[h][0], r1 = f.xa[h][1];
-    const uint32_t a_s0[4] = {r0.x, r1.x, r0.y, r1.y};
-    const uint32_t a_s1[4] = {r0.z, r1.z, r0.w, r1.w};
+  for (int L = 0; L < LOG2; L++) {
+    if ((i >> L) & 1) {
 #pragma unroll
-    for (int t = 0; t < NT; t++) {
-      const uint4 b = f.ab[h][t];
-      const uint32_t b_s0[2] = {b.x, b.y};
-      const uint32_t b_s1[2] = {b.z, b.w};
-      mma_bf16_16816(acc[t], a_s0, b_s0, acc[t]);
-      mma_bf16_16816(acc[t], a_s1, b_s1, acc[t]);
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) acc[t][q] = __fadd_rn(lv[L][t][q], acc[t][q]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) lv[L][t][q] = acc[t][q];
+      break;
     }
+  }
+}
+
+// Warp 0 of a CTA: its row tile's adapter (-1: no tile, n_ad: tokens
+// without an adapter), rows, and the token index of each row, into shared
+// memory.  With a plan, one read of the tile's table record (the CTA tile
+// is part q of record tile / sub); without one, rows in index order.
+BI_DEV void tile_record(const ShrinkParams &p, int bm, int tile, int lane, int32_t *s_rows, int *s_info) {
+  int adapter = -1, rows = 0;
+  if (p.table) {
+    const int rec = tile / p.sub, q = tile - rec * p.sub;
+    const int32_t *R = p.table + (size_t)rec * kPlanRec;
+    const int4 h = *reinterpret_cast<const int4 *>(R);
+    int4 id4 = make_int4(0, 0, 0, 0);
+    if (lane < kPlanTile / 4) id4 = *reinterpret_cast<const int4 *>(R + 4 + 4 * lane);
+    rows = min(bm, h.y - q * bm);
+    adapter = rows > 0 ? h.x : -1;
+    const int idv[4] = {id4.x, id4.y, id4.z, id4.w};
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int s = 4 * lane + e - q * bm;
+      if (lane < kPlanTile / 4 && s >= 0 && s < rows) s_rows[s] = idv[e];
+    }
+  } else {
+    const int row0 = tile * bm;
+    rows = min(bm, p.M - row0);
+    adapter = rows > 0 ? 0 : -1;
+    for (int i = lane; i < rows; i += 32) s_rows[i] = row0 + i;
+  }
+  if (lane == 0) {
+    s_info[0] = adapter;
+    s_info[1] = rows > 0 ? rows : 0;
+  }
+}
+
+// The G group values of a row tile (part [G][bm][r], in shared memory,
+// written and visible to the CTA) -> the tile's y rows: the perfect tree over
+// the groups, then the cross-split combine of the mode.  Every thread of the
+// CTA calls it.  In mode TREE with splits > 1 each CTA has made a relaxed
+// cluster arrive on entry; the matching wait comes before the first write
+// into a peer's shared memory.  slots: the exchange slots (mode TREE).
+BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const int32_t *s_rows,
+                        int rows, int bm, int split) {
+  const int E = bm * p.r;
+  const int r_sh = (p.r & (p.r - 1)) == 0 ? __ffs(p.r) - 1 : -1;
+  auto e_row = [&](int e) { return r_sh >= 0 ? e >> r_sh : e / p.r; };
+  auto e_col = [&](int e) { return r_sh >= 0 ? e & (p.r - 1) : e % p.r; };
+  // perfect tree over the G groups, in place into group 0
+  for (int s = 1; s < p.groups; s <<= 1) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      for (int q = 0; q + s < p.groups; q += 2 * s)
+        part[(size_t)q * E + e] = __fadd_rn(part[(size_t)q * E + e], part[(size_t)(q + s) * E + e]);
+    __syncthreads();
+  }
+
+  auto out_index = [&](int e) -> size_t { return (size_t)s_rows[e_row(e)] * p.r + e_col(e); };
+  const int valid_E = rows * p.r;
+
+  if (p.mode == BI_SHRINK_ATOMIC) {
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) atomicAdd(p.y + out_index(e), part[e]);
+    return;
+  }
+  if (p.splits == 1) {
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) p.y[out_index(e)] = part[e];
+    return;
+  }
+
+  // ---- mode TREE: the splits CTAs of this tile form one cluster; rank q
+  // holds the subtree of leaves [q*lc, (q+1)*lc).  The tile's E elements
+  // are cut into S shares; rank q finishes share q.  Before one cluster
+  // barrier every rank stores share t of its partial into rank t's slot
+  // [q] through distributed shared memory (a reduce-scatter by pushes);
+  // after it (release / acquire) each rank adds the S values of its share
+  // by the perfect tree over the ranks, from its own shared memory, and
+  // writes y.  Nothing reads a peer's memory after the barrier, so one
+  // barrier is enough, and every SM receives only (S-1)/S of one partial.
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = p.splits;
+  // the relaxed arrive each CTA made on entry: once this wait returns,
+  // every CTA of the cluster is running, so its shared memory may be written
+  cluster_wait();
+  if (p.gather0) {
+    // small tiles: ranks 1..S-1 push their whole partial into rank 0's
+    // slots [S-1][E]; after the barrier rank 0 alone adds and writes y
+    float *gslots = slots;
+    if (split != 0) {
+      float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(gslots, 0) + (size_t)(split - 1) * E);
+      const float4 *src = reinterpret_cast<const float4 *>(part);
+      for (int e4 = threadIdx.x; e4 < E / 4; e4 += blockDim.x) dst[e4] = src[e4];
+    }
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (split != 0) return;
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
+      float v[kMaxSplits];
+      v[0] = part[e];
+#pragma unroll
+      for (int q = 1; q < kMaxSplits; q++) v[q] = q < S ? gslots[(size_t)(q - 1) * E + e] : 0.0f;
+#pragma unroll
+      for (int st = 1; st < kMaxSplits; st <<= 1)
+#pragma unroll
+        for (int q = 0; q + st < kMaxSplits; q += 2 * st)
+          if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
+      p.y[out_index(e)] = v[0];
+    }
+    return;
+  }
+  const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
+  for (int t = 0; t < S; t++) {
+    if (t == split) continue;
+    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
+    const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
+    for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  for (int i = threadIdx.x; i < share; i += blockDim.x) {
+    const int e = split * share + i;
+    if (e >= valid_E) break;
+    float v[kMaxSplits];
+#pragma unroll
+    for (int q = 0; q < kMaxSplits; q++)
+      v[q] = q < S ? (q == split ? part[e] : slots[(size_t)q * share + i]) : 0.0f;
+#pragma unroll
+    for (int st = 1; st < kMaxSplits; st <<= 1)
+#pragma unroll
+      for (int q = 0; q + st < kMaxSplits; q += 2 * st)
+        if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
+    p.y[out_index(e)] = v[0];
   }
 }
 
@@ -111,18 +295,26 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   constexpr int NT = NGW / 8;
   extern __shared__ float4 smem_f4[];
   float *part = reinterpret_cast<float *>(smem_f4);     // [G][BM][r]
-  __shared__ TileInfo s_tile;
-  __shared__ int32_t s_off[kMaxAdapters + 2];
   __shared__ int32_t s_rows[kMaxBM];                    // token row of each tile row
+  __shared__ int s_info[2];
 
   const int bm = 16 * p.mtiles;
   const int split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
 
-  resolve_tile_block(p.offsets, p.n_ad, p.M, blockIdx.y, bm, s_off, &s_tile);
-  const TileInfo ti = s_tile;
-  if (ti.adapter < 0) return;                       // uniform across the cluster
+  if (warp == 0) tile_record(p, bm, blockIdx.y, lane, s_rows, s_info);
+  __syncthreads();
+  struct { int adapter, rows; } ti = {s_info[0], s_info[1]};
+  // mode TREE: say "started" to the cluster now; finish_tile waits for the
+  // others before it writes into their shared memory.  The exits below are
+  // uniform across the cluster (every split sees the same tile) and wait too.
+  const bool clustered = p.mode == BI_SHRINK_TREE && p.splits > 1;
+  if (clustered) cluster_arrive_relaxed();
+  if (ti.adapter < 0) {
+    if (clustered) cluster_wait();
+    return;
+  }
 
   // e -> (local row, column) of the [bm][r] tile; r is a power of two in
   // every common configuration, so the split is a shift and a mask
@@ -131,15 +323,12 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   auto e_col = [&](int e) { return r_sh >= 0 ? e & (p.r - 1) : e % p.r; };
 
   if (ti.adapter == p.n_ad) {                       // tokens without an adapter
-    if (p.mode != BI_SHRINK_ATOMIC && split == 0) {
-      for (int e = threadIdx.x; e < ti.rows * p.r; e += blockDim.x) {
-        const int pos = ti.seg_begin + ti.row0 + e_row(e);
-        p.y[(size_t)p.perm[pos] * p.r + e_col(e)] = 0.0f;
-      }
-    }
+    if (p.mode != BI_SHRINK_ATOMIC && split == 0)
+      for (int e = threadIdx.x; e < ti.rows * p.r; e += blockDim.x)
+        p.y[(size_t)s_rows[e_row(e)] * p.r + e_col(e)] = 0.0f;
+    if (clustered) cluster_wait();
     return;
   }
-  if ((int)threadIdx.x < ti.rows) s_rows[threadIdx.x] = tile_row(p.perm, ti, threadIdx.x);
 
   // ---- warp role: (leaf group, m-tile, rank group)
   const int per_lg = p.mtiles * p.ngroups;
@@ -154,8 +343,8 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   // token rows of this thread's fragment rows: their loads go out before
   // the A staging, since the x loads wait on them
   int row0 = 0, row1 = 0;
-  if (v0) row0 = tile_row(p.perm, ti, lr0);
-  if (v1) row1 = tile_row(p.perm, ti, lr1);
+  if (v0) row0 = s_rows[lr0];
+  if (v1) row1 = s_rows[lr1];
 
   // ---- shared memory holds the CTA's A slice (staged once, by every
   // thread with 16-byte cp.async, when it fits in 64 KB).  Rows are 128 bytes
@@ -228,38 +417,32 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   }
 
   if constexpr (LG > 0) {
-    // binary counter: leaf i closes the levels where its index has a 1 bit
-    // (left = the parked subtree, right = the one just finished) and parks
-    // the result at its lowest 0 bit; every index is a compile-time constant
+    // binary counter over the group's leaves (every index a compile-time
+    // constant), two leaves' MMAs interleaved when the ring allows it
     constexpr int LOG2 = LG >= 16 ? 4 : (LG >= 8 ? 3 : (LG >= 4 ? 2 : (LG >= 2 ? 1 : 0)));
+    constexpr int NB = (LG >= 2 && PF % 2 == 0) ? 2 : 1;
     float lv[LOG2 > 0 ? LOG2 : 1][NT][4];
 #pragma unroll
-    for (int i = 0; i < LG; i++) {
-      LeafFrag<NT> f = ring[i % PF];
-      if (i + PF < LG) load_leaf(ring[i % PF], leaf0 + i + PF);
-      a_frags(f, i);
-      float acc[NT][4];
-      mma_leaf<NT>(acc, f);
+    for (int i0 = 0; i0 < LG; i0 += NB) {
+      LeafFrag<NT> f[NB];
 #pragma unroll
-      for (int L = 0; L < LOG2; L++) {
-        if ((i >> L) & 1) {
-#pragma unroll
-          for (int t = 0; t < NT; t++)
-#pragma unroll
-            for (int q = 0; q < 4; q++) acc[t][q] = __fadd_rn(lv[L][t][q], acc[t][q]);
-        } else {
-#pragma unroll
-          for (int t = 0; t < NT; t++)
-#pragma unroll
-            for (int q = 0; q < 4; q++) lv[L][t][q] = acc[t][q];
-          break;
-        }
+      for (int b = 0; b < NB; b++) {
+        const int i = i0 + b;
+        f[b] = ring[i % PF];
+        if (i + PF < LG) load_leaf(ring[i % PF], leaf0 + i + PF);
+        a_frags(f[b], i);
       }
-      if (i == LG - 1)
+      float acc[NB][NT][4];
+      mma_leaves<NT, NB>(acc, f);
 #pragma unroll
-        for (int t = 0; t < NT; t++)
+      for (int b = 0; b < NB; b++) {
+        fold_leaf<NT, LOG2>(i0 + b, lv, acc[b]);
+        if (i0 + b == LG - 1)
 #pragma unroll
-          for (int q = 0; q < 4; q++) res[t][q] = acc[t][q];
+          for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) res[t][q] = acc[b][t][q];
+      }
     }
   } else {
     float st[MAXD][NT][4];
@@ -328,87 +511,193 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
     *reinterpret_cast<float2 *>(dst + lr1 * p.r + col) = make_float2(res[t][2], res[t][3]);
   }
   __syncthreads();
-  // perfect tree over the G groups, in place into group 0
-  for (int s = 1; s < p.groups; s <<= 1) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-      for (int q = 0; q + s < p.groups; q += 2 * s)
-        part[(size_t)q * E + e] = __fadd_rn(part[(size_t)q * E + e], part[(size_t)(q + s) * E + e]);
-    __syncthreads();
+  float *slots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);
+  finish_tile(p, part, slots, s_rows, ti.rows, bm, split);
+}
+
+// ----------------------------------------------------------------------
+// Bulk-copy kernel: the CTA's whole x slice (bm rows x lc leaves) and,
+// when staged, its A slice (r rows x lc leaves) are requested from HBM by
+// the copy engine as soon as the tile is known, one contiguous
+// `cp.async.bulk` per row (rowbytes = lc * 128 bytes), so a CTA has every
+// byte it needs in flight after two dependent reads (its table record,
+// then x).  Each 16-row m-tile lands on its own mbarrier; its warps start
+// multiplying as soon as their rows are in.  Used when the slice fits:
+// lc <= 16 leaves per split (e.g. K = 4096 at splits >= 4).
+//
+// Shared memory: [0, 64) mbarriers (m-tiles 0..3, A = 4); [64, 320) token
+// rows; [320, 328) adapter and rows; x rows at x_off (row stride rowbytes);
+// A rows at a_offset; the group values at part_off (they may overlay the x
+// rows, which are dead by then); the TREE exchange slots at g_offset.
+//
+// Fragment reads: threads (g, c) of an 8-lane phase read rows g = 2q and
+// 2q + 1.  Rows are rowbytes apart (a multiple of 128), so the same 64-byte
+// half of both rows would fall on the same banks; odd rows therefore read
+// their two halves in the other order, which makes every phase
+// conflict-free without padding.
+// ----------------------------------------------------------------------
+template <int NGW, int LG, bool ASTAGED>
+__global__ void __launch_bounds__(256)
+shrink_bulk_kernel(const __grid_constant__ ShrinkParams p) {
+  constexpr int NT = NGW / 8;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+  int32_t *s_rows = reinterpret_cast<int32_t *>(smem + 64);
+  int *s_info = reinterpret_cast<int *>(smem + 320);
+  constexpr int kABar = 4;
+
+  const int bm = 16 * p.mtiles;
+  const int split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
+
+  // ---- the tile: adapter, rows and their token indices (one read)
+  if (warp == 0) tile_record(p, bm, blockIdx.y, lane, s_rows, s_info);
+  if (warp == (nwarps > 1 ? 1 : 0) && lane == 0) {
+#pragma unroll
+    for (int i = 0; i <= kABar; i++) mbar_init(&bars[i], 1);
+    mbar_fence_init();
   }
-
-  auto out_index = [&](int e) -> size_t { return (size_t)s_rows[e_row(e)] * p.r + e_col(e); };
-  const int valid_E = ti.rows * p.r;
-
-  if (p.mode == BI_SHRINK_ATOMIC) {
-    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) atomicAdd(p.y + out_index(e), part[e]);
+  __syncthreads();
+  const int adapter = s_info[0], rows = s_info[1];
+  const bool clustered = p.mode == BI_SHRINK_TREE && p.splits > 1;
+  if (clustered) cluster_arrive_relaxed();          // matched in finish_tile / below
+  if (adapter < 0) {                                // uniform across the cluster
+    if (clustered) cluster_wait();
     return;
   }
-  if (p.splits == 1) {
-    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) p.y[out_index(e)] = part[e];
+  if (adapter == p.n_ad) {                          // tokens without an adapter
+    if (p.mode != BI_SHRINK_ATOMIC && split == 0)
+      for (int e = threadIdx.x; e < rows * p.r; e += blockDim.x) p.y[(size_t)s_rows[e / p.r] * p.r + e % p.r] = 0.0f;
+    if (clustered) cluster_wait();
     return;
   }
 
-  // ---- mode TREE: the splits CTAs of this tile form one cluster; rank q
-  // holds the subtree of leaves [q*lc, (q+1)*lc).  The tile's E elements
-  // are cut into S shares; rank q finishes share q.  Before one cluster
-  // barrier every rank stores share t of its partial into rank t's slot
-  // [q] through distributed shared memory (a reduce-scatter by pushes);
-  // after it (release / acquire) each rank adds the S values of its share
-  // by the perfect tree over the ranks, from its own shared memory, and
-  // writes y.  Nothing reads a peer's memory after the barrier, so one
-  // barrier is enough, and every SM receives only (S-1)/S of one partial.
-  cg::cluster_group cluster = cg::this_cluster();
-  const int S = p.splits;
-  if (p.gather0) {
-    // small tiles: ranks 1..S-1 push their whole partial into rank 0's
-    // slots [S-1][E]; after the barrier rank 0 alone adds and writes y
-    float *gslots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);
-    if (split != 0) {
-      float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(gslots, 0) + (size_t)(split - 1) * E);
-      const float4 *src = reinterpret_cast<const float4 *>(part);
-      for (int e4 = threadIdx.x; e4 < E / 4; e4 += blockDim.x) dst[e4] = src[e4];
+  // ---- every byte of the slice requested at once
+  uint8_t *xs = smem + p.x_off;
+  uint8_t *as = smem + p.a_offset;
+  const uint32_t rb = (uint32_t)p.rowbytes;
+  const size_t row_bytes = (size_t)p.K * 2;
+  const size_t koff = (size_t)split * rb;           // this split's K range inside a row
+  if (warp < p.mtiles) {
+    const int nv = max(0, min(16, rows - 16 * warp));
+    if (lane == 0) mbar_arrive_expect_tx(&bars[warp], (uint32_t)nv * rb);
+    __syncwarp();
+    if (lane < nv)
+      bulk_load(xs + (size_t)(16 * warp + lane) * rb,
+                reinterpret_cast<const uint8_t *>(p.x) + (size_t)s_rows[16 * warp + lane] * row_bytes + koff, rb,
+                &bars[warp]);
+  }
+  if (ASTAGED && warp == (nwarps > p.mtiles ? p.mtiles : 0)) {
+    if (lane == 0) mbar_arrive_expect_tx(&bars[kABar], (uint32_t)p.r * rb);
+    __syncwarp();
+    for (int j = lane; j < p.r; j += 32)
+      bulk_load(as + (size_t)j * rb,
+                reinterpret_cast<const uint8_t *>(p.at) + ((size_t)adapter * p.r + j) * row_bytes + koff, rb,
+                &bars[kABar]);
+  }
+
+  // ---- warp role: (leaf group, m-tile, rank group)
+  const int per_lg = p.mtiles * p.ngroups;
+  const int lgi = warp / per_lg;
+  const int mt = (warp % per_lg) / p.ngroups;
+  const int ng = warp % p.ngroups;
+  const int lr0 = mt * 16 + g, lr1 = lr0 + 8;
+
+  // A fragments straight from global memory (L2) when A is not staged
+  const uint16_t *acol[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+    acol[t] = p.at + ((size_t)adapter * p.r + ng * NGW + t * 8 + g) * p.K + (size_t)split * p.lc * kLeaf +
+              (size_t)lgi * LG * kLeaf + 8 * c;
+  LeafFrag<NT> agl[ASTAGED ? 1 : LG];
+  if (!ASTAGED) {
+#pragma unroll
+    for (int i = 0; i < LG; i++)
+#pragma unroll
+      for (int h = 0; h < 2; h++)
+#pragma unroll
+        for (int t = 0; t < NT; t++) agl[ASTAGED ? 0 : i].ab[h][t] = ldg128(acol[t] + i * kLeaf + 32 * h);
+  }
+
+  bool ok = mbar_wait(&bars[mt], 0);
+  if (ASTAGED) ok = mbar_wait(&bars[kABar], 0) && ok;
+  if (!ok) flag_error(p.status, BI_ERR_TIMEOUT);
+
+  const int odd = g & 1;
+  const int hA = odd ? 64 : 0, hB = 64 - hA;
+  const uint8_t *xr0 = xs + (size_t)lr0 * rb + c * 16;
+  const uint8_t *xr1 = xr0 + (size_t)8 * rb;
+  auto lds = [](const uint8_t *q) { return *reinterpret_cast<const uint4 *>(q); };
+
+  float res[NT][4];
+  {
+    constexpr int LOG2 = LG >= 16 ? 4 : (LG >= 8 ? 3 : (LG >= 4 ? 2 : (LG >= 2 ? 1 : 0)));
+    constexpr int NB = LG < 4 ? LG : 4;             // leaves whose MMAs are interleaved
+    float lv[LOG2 > 0 ? LOG2 : 1][NT][4];
+#pragma unroll
+    for (int i0 = 0; i0 < LG; i0 += NB) {
+      LeafFrag<NT> f[NB];
+#pragma unroll
+      for (int b = 0; b < NB; b++) {
+        const int i = i0 + b;
+        const int lb = (lgi * LG + i) * 128;
+        const uint4 p0 = lds(xr0 + lb + hA), p1 = lds(xr0 + lb + hB);
+        const uint4 q0 = lds(xr1 + lb + hA), q1 = lds(xr1 + lb + hB);
+        f[b].xa[0][0] = odd ? p1 : p0;
+        f[b].xa[1][0] = odd ? p0 : p1;
+        f[b].xa[0][1] = odd ? q1 : q0;
+        f[b].xa[1][1] = odd ? q0 : q1;
+        if (ASTAGED) {
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            const uint8_t *ar = as + (size_t)(ng * NGW + t * 8 + g) * rb + c * 16 + lb;
+            const uint4 a0 = lds(ar + hA), a1 = lds(ar + hB);
+            f[b].ab[0][t] = odd ? a1 : a0;
+            f[b].ab[1][t] = odd ? a0 : a1;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; h++)
+#pragma unroll
+            for (int t = 0; t < NT; t++) f[b].ab[h][t] = agl[ASTAGED ? 0 : i].ab[h][t];
+        }
+      }
+      float acc[NB][NT][4];
+      mma_leaves<NT, NB>(acc, f);
+#pragma unroll
+      for (int b = 0; b < NB; b++) {
+        fold_leaf<NT, LOG2>(i0 + b, lv, acc[b]);
+        if (i0 + b == LG - 1)
+#pragma unroll
+          for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) res[t][q] = acc[b][t][q];
+      }
     }
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    if (split != 0) return;
-    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
-      float v[kMaxSplits];
-      v[0] = part[e];
-#pragma unroll
-      for (int q = 1; q < kMaxSplits; q++) v[q] = q < S ? gslots[(size_t)(q - 1) * E + e] : 0.0f;
-#pragma unroll
-      for (int st = 1; st < kMaxSplits; st <<= 1)
-#pragma unroll
-        for (int q = 0; q + st < kMaxSplits; q += 2 * st)
-          if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
-      p.y[out_index(e)] = v[0];
-    }
-    return;
   }
-  const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
-  float *slots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);  // [S][share]
-  for (int t = 0; t < S; t++) {
-    if (t == split) continue;
-    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
-    const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
-    for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
+  if (!ok) {
+    // a copy may still be landing: wait for it (bounded) before the rows'
+    // space is reused or the CTA exits
+    mbar_wait(&bars[mt], 0);
+    if (ASTAGED) mbar_wait(&bars[kABar], 0);
   }
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  for (int i = threadIdx.x; i < share; i += blockDim.x) {
-    const int e = split * share + i;
-    if (e >= valid_E) break;
-    float v[kMaxSplits];
+  __syncthreads();                                  // every warp is done with the x rows
+
+  // ---- group values -> shared memory (over the x rows), then the combine
+  float *part = reinterpret_cast<float *>(smem + p.part_off);
+  const int E = bm * p.r;
 #pragma unroll
-    for (int q = 0; q < kMaxSplits; q++)
-      v[q] = q < S ? (q == split ? part[e] : slots[(size_t)q * share + i]) : 0.0f;
-#pragma unroll
-    for (int st = 1; st < kMaxSplits; st <<= 1)
-#pragma unroll
-      for (int q = 0; q + st < kMaxSplits; q += 2 * st)
-        if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
-    p.y[out_index(e)] = v[0];
+  for (int t = 0; t < NT; t++) {
+    const int col = ng * NGW + t * 8 + 2 * c;
+    float *dst = part + (size_t)lgi * E;
+    *reinterpret_cast<float2 *>(dst + lr0 * p.r + col) = make_float2(res[t][0], res[t][1]);
+    *reinterpret_cast<float2 *>(dst + lr1 * p.r + col) = make_float2(res[t][2], res[t][3]);
   }
+  __syncthreads();
+  float *slots = reinterpret_cast<float *>(smem + p.g_offset);
+  finish_tile(p, part, slots, s_rows, rows, bm, split);
 }
 
 // ----------------------------------------------------------------------
@@ -470,10 +759,103 @@ static cudaError_t launch_shrink_t(const ShrinkParams &p, int tiles, int threads
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-// Validates, picks the (bit-neutral) tiling and launches.  perm/offsets are
-// null for the single-adapter call.
+static cudaError_t launch_bulk(void (*kern)(ShrinkParams), const ShrinkParams &p, int tiles, int threads, size_t smem,
+                               cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, tiles, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  int na = 0;
+  if (p.mode == BI_SHRINK_TREE && p.splits > 1) {
+    if (p.splits > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    na = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int NGW, bool ASTAGED>
+static void (*bulk_kernel_for(int lg))(ShrinkParams) {
+  switch (lg) {
+    case 1: return shrink_bulk_kernel<NGW, 1, ASTAGED>;
+    case 2: return shrink_bulk_kernel<NGW, 2, ASTAGED>;
+    case 4: return shrink_bulk_kernel<NGW, 4, ASTAGED>;
+    default:
+      if constexpr (ASTAGED) {
+        if (lg == 8) return shrink_bulk_kernel<NGW, 8, true>;
+        if (lg == 16) return shrink_bulk_kernel<NGW, 16, true>;
+      }
+      return nullptr;
+  }
+}
+
+static void (*bulk_kernel(int ngw, bool staged, int lg))(ShrinkParams) {
+  if (ngw == 16) return staged ? bulk_kernel_for<16, true>(lg) : bulk_kernel_for<16, false>(lg);
+  return staged ? bulk_kernel_for<8, true>(lg) : bulk_kernel_for<8, false>(lg);
+}
+
+// Tiling of the bulk-copy kernel (bit-neutral), or false when the slice does
+// not fit it: up to four 16-row m-tiles (at most 64 KB of x rows), then
+// leaf groups until the CTA has eight warps; A staged in shared memory when
+// its slice is at most 64 KB, else read from L2 by the warps (then at most
+// four leaves per warp, their A fragments held in registers).
+static bool bulk_tiling(ShrinkParams &p, int M, bool segmented, int &threads, int &tiles, size_t &smem) {
+  const int rb = p.lc * 128;
+  if (16 * rb > 64 * 1024) return false;
+  int mt = std::min(4, (M + 15) / 16);
+  while (mt > 1 && (mt * p.ngroups > 8 || 16 * mt * rb > 64 * 1024)) mt >>= 1;
+  int G = 1;
+  while (p.lc % (2 * G) == 0 && 2 * G * mt * p.ngroups <= 8) G *= 2;
+  const int lg = p.lc / G;
+  if (lg != 1 && lg != 2 && lg != 4 && lg != 8 && lg != 16) return false;
+  const size_t a_bytes = (size_t)p.r * rb;
+  const bool staged = a_bytes <= 64 * 1024;
+  if (!staged && lg > 4) return false;
+  const int bm = 16 * mt;
+  p.mtiles = mt;
+  p.groups = G;
+  p.lg = lg;
+  p.a_staged = staged ? 1 : 0;
+  p.rowbytes = rb;
+  p.sub = kPlanTile / bm;
+  p.x_off = 512;
+  size_t off = (size_t)p.x_off + (size_t)bm * rb;
+  p.a_offset = (int)off;
+  if (staged) off += a_bytes;
+  const size_t part_bytes = (size_t)G * bm * p.r * sizeof(float);
+  if (part_bytes <= (size_t)bm * rb) {
+    p.part_off = p.x_off;
+  } else {
+    p.part_off = (int)off;
+    off += part_bytes;
+  }
+  const size_t part1 = (size_t)bm * p.r * sizeof(float);
+  p.gather0 = p.mode == BI_SHRINK_TREE && p.splits > 1 && (size_t)(p.splits - 1) * part1 <= 8 * 1024 ? 1 : 0;
+  off = (off + 127) & ~size_t(127);
+  p.g_offset = (int)off;
+  if (p.mode == BI_SHRINK_TREE && p.splits > 1) off += p.gather0 ? (size_t)(p.splits - 1) * part1 : part1;
+  smem = off;
+  threads = 32 * G * mt * p.ngroups;
+  tiles = segmented ? (int)plan_tiles(M, p.n_ad) * p.sub : (M + bm - 1) / bm;
+  return smem <= 200 * 1024;
+}
+
+// Validates, picks the kernel and its (bit-neutral) tiling and launches.
+// perm / offsets / table are null for the single-adapter call.
 bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const int32_t *offsets,
-                        int n_ad, float *y, int M, int K, int r, int splits, int mode,
+                        const int32_t *table, int n_ad, float *y, int M, int K, int r, int splits, int mode,
                         cudaStream_t stream) {
   if (M < 0 || K <= 0 || r <= 0 || n_ad < 1) return BI_ERR_INVALID_ARG;
   if (mode != BI_SHRINK_UNSPLIT && mode != BI_SHRINK_ATOMIC && mode != BI_SHRINK_TREE)
@@ -491,6 +873,7 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   p.at = static_cast<const uint16_t *>(A);
   p.perm = perm;
   p.offsets = offsets;
+  p.table = table;
   p.y = y;
   p.status = status_word();
   p.M = M; p.K = K; p.r = r; p.n_ad = n_ad;
@@ -500,10 +883,29 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
 
   const int ngw = (r % 16 == 0) ? 16 : 8;
   p.ngroups = r / ngw;
+  if (p.ngroups > 8) return BI_ERR_UNSUPPORTED_SHAPE;
+
+  {
+    ShrinkParams q = p;
+    int threads = 0, tiles = 0;
+    size_t smem = 0;
+    void (*kern)(ShrinkParams) = nullptr;
+    if (bulk_tiling(q, M, table != nullptr, threads, tiles, smem)) kern = bulk_kernel(ngw, q.a_staged != 0, q.lg);
+    // The bulk kernel has every CTA request its whole slice at once, which
+    // wins while the grid is resident in one wave (measured: M = 1024 at
+    // split-K 8 in 7.3 us against 9-10 us); beyond that its 64 KB of x per
+    // CTA halves the CTAs per SM and the register-ring kernel streams faster.
+    int per_sm = 0;
+    if (kern && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) == cudaSuccess &&
+        (long)tiles * splits * (splits > 1 && mode == BI_SHRINK_TREE ? 8 : 7) <= 7L * per_sm * num_sms()) {
+      if (mode == BI_SHRINK_ATOMIC) BI_CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)M * r * sizeof(float), stream));
+      return launch_bulk(kern, q, tiles, threads, smem, stream) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    }
+  }
   // Tiling (bit-neutral).  Leaf groups first: enough warps per row tile
   // that each walks at most 8 leaves (a power of two dividing the split's
   // leaves); then up to 4 row tiles of 16, at most 8 warps per CTA.
-  if (p.ngroups > 8) return BI_ERR_UNSUPPORTED_SHAPE;
   int G = 1;
   while (p.lc / G > 8 && p.lc % (G * 2) == 0 && G * 2 * p.ngroups <= 8) G *= 2;
   int mt = std::min(4, (M + 15) / 16);
@@ -537,7 +939,8 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   const size_t base_smem = part_bytes + (p.a_staged ? a_bytes : 0);
   p.g_offset = (int)base_smem;
   const size_t smem = base_smem + slot_bytes;
-  const int tiles = offsets ? (M + bm - 1) / bm + n_ad + 1 : (M + bm - 1) / bm;
+  p.sub = kPlanTile / bm;
+  const int tiles = table ? (int)plan_tiles(M, n_ad) * p.sub : (M + bm - 1) / bm;
 
   if (mode == BI_SHRINK_ATOMIC) {
     BI_CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)M * r * sizeof(float), stream));
@@ -567,7 +970,7 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
 
 extern "C" bi_status bi_lora_shrink(const void *x, const void *A, float *y, int M, int K, int r,
                                     int splits, int mode, bi_stream_t stream) {
-  return bi::shrink_launch(x, A, nullptr, nullptr, 1, y, M, K, r, splits, mode,
+  return bi::shrink_launch(x, A, nullptr, nullptr, nullptr, 1, y, M, K, r, splits, mode,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -575,9 +978,11 @@ extern "C" bi_status bi_lora_shrink_segmented(const void *x, const void *A, cons
                                               int n_adapters, float *y, int M, int K, int r,
                                               int splits, int mode, bi_stream_t stream) {
   if (M > 0 && !plan) return BI_ERR_INVALID_ARG;
-  if (n_adapters < 1 || n_adapters > 256) return BI_ERR_INVALID_ARG;
+  if (n_adapters < 1 || n_adapters > bi::kMaxAdapters) return BI_ERR_INVALID_ARG;
+  if (M > 0 && !bi_aligned16(plan)) return BI_ERR_UNSUPPORTED_SHAPE;
   const int32_t *perm = static_cast<const int32_t *>(plan);
   const int32_t *offsets = perm + M;
-  return bi::shrink_launch(x, A, perm, offsets, n_adapters, y, M, K, r, splits, mode,
+  const int32_t *table = perm + bi::plan_table_word(M, n_adapters);
+  return bi::shrink_launch(x, A, perm, offsets, table, n_adapters, y, M, K, r, splits, mode,
                            reinterpret_cast<cudaStream_t>(stream));
 }

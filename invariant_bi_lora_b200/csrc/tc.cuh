@@ -79,6 +79,31 @@ BI_DEV void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x,
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// Contiguous bulk copy global -> this CTA's shared memory by the copy
+// engine, completion counted on `bar` (bytes).  No multicast.  Both
+// addresses 16-byte aligned, `bytes` a multiple of 16.
+BI_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// The same with an L2 eviction-priority hint (`policy` from createpolicy).
+BI_DEV void bulk_load_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// L2 policy for data read exactly once: evict it first.
+BI_DEV uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // Per-thread 16-byte asynchronous copy global -> shared (LDGSTS, L2 only),
 // and an arrival on `bar` that fires once all of this thread's earlier
 // cp.async copies have landed (the barrier's count must include it: noinc).
@@ -179,6 +204,5 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
 // library does not link libcuda directly.
 bool make_tma_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer);
-int num_sms();
 
 }  // namespace bi

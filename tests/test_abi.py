@@ -36,8 +36,11 @@ def test_status_strings(libbi):
 
 def test_sizes(libbi):
     from invariant_bi_lora_b200 import bi
-    assert bi.lora_plan_bytes(4096, 8) == 4 * (4096 + 10)
-    assert bi.lora_plan_bytes(0, 1) == 4 * 3
+    from helpers import plan_words
+    # perm 4096 + offsets 10 + 2 words of padding + 73 records of 68 words
+    assert bi.lora_plan_bytes(4096, 8) == 4 * (4096 + 10 + 2 + 68 * 73) == 4 * plan_words(4096, 8)
+    assert bi.lora_plan_bytes(0, 1) == 4 * (4 + 68 * 2) == 4 * plan_words(0, 1)
+    assert bi.lora_plan_bytes(1000, 256) == 4 * plan_words(1000, 256)
 
 
 FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: every call below fails validation
@@ -63,6 +66,7 @@ def test_other_rejects(libbi):
     assert libbi.bi_lora_shrink(ctypes.c_void_p(0x10001), FAKE, FAKE, 4, 64, 8, 1, 0, None) == 2  # misaligned
     assert libbi.bi_lora_plan(FAKE, 16, 0, FAKE, 1 << 20, None) == 1
     assert libbi.bi_lora_plan(FAKE, 16, 8, FAKE, 8, None) == 3                   # plan too small
+    assert libbi.bi_lora_plan(FAKE, 16, 8, ctypes.c_void_p(0x10004), 1 << 20, None) == 2   # not 16-byte aligned
     assert libbi.bi_lora_expand(FAKE, FAKE, FAKE, 4, 12, 64, 0, None) == 2
     assert libbi.bi_rmsnorm(FAKE, FAKE, FAKE, 4, 100, ctypes.c_float(1e-6), None) == 2
     assert libbi.bi_log_softmax(FAKE, FAKE, 4, 6, None) == 2

@@ -62,14 +62,15 @@ def test_gemm_bf16_output():
 
 @pytest.mark.parametrize("N", [4096, 14336])
 def test_gemm_batch_invariance(N):
-    """Rows of the M=1 result == the same rows at M = 16, 64, 256, 1024, 4096
-    (K=4096), wherever they sit in a tile."""
+    """Rows of the M=1 result == the same rows at M = 16 ... 4096 (K=4096),
+    wherever they sit in a tile; the M values cross the tile-width changes
+    (128 x 32 up to M = 128, 128 x 64 up to 512, 128 x 256 above)."""
     K = 4096
     big_a, w = synth.gemm_inputs(4096, N, K, seed=7)
     W = dev_bf16(w)
     probe = big_a[:8]
     ref = np.stack([host_bits(run_gemm(dev_bf16(probe[i:i + 1]), W))[0] for i in range(8)])
-    for M in (16, 64, 256, 1024, 4096):
+    for M in (16, 64, 128, 129, 256, 512, 513, 1024, 4096):
         a = big_a[:M].copy()
         positions = sorted({0, M - 1, min(127, M - 1), min(128, M - 1), M // 2, max(0, M - 8)})
         for j, pos in enumerate(positions):
@@ -98,3 +99,27 @@ def test_gemm_rejects():
     C = torch.empty(0, 16, dtype=torch.float32, device="cuda")
     bi.gemm(torch.empty(0, 64, dtype=torch.bfloat16, device="cuda"),
             dev_bf16(synth.normal_bf16((16, 64), 1.0, seed=1)), C)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (64, 512, 1024), (300, 1040, 1024), (1024, 4096, 4096)])
+def test_addmm(M, N, K):
+    """torch.addmm ("Batch Invariant Ops", Highlighted Details): within
+    tolerance of the oracle's exact bias + A.W^T, and bitwise the GEMM's fp32
+    result plus the bias in one IEEE addition (bf16 output: its RNE)."""
+    a, w = synth.gemm_inputs(M, N, K, seed=M + 5)
+    bias = synth.normal_bf16((N,), 1.0, seed=M, tag=9)
+    A, W, Bv = dev_bf16(a), dev_bf16(w), dev_bf16(bias)
+    C = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    bi.addmm(Bv, A, W, C)
+    G = run_gemm(A, W)
+    assert torch.equal(C.view(torch.int32), (G + Bv.float()[None, :]).view(torch.int32))
+    C16 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    bi.addmm(Bv, A, W, C16)
+    assert torch.equal(C16.view(torch.int16), C.to(torch.bfloat16).view(torch.int16))
+    rows = np.unique(np.concatenate([np.arange(min(M, 24)), np.arange(max(0, M - 24), M)]))
+    exact, bound = oracle.addmm_exact(bias, a, w, rows=rows)
+    assert_tol(C.cpu().numpy()[rows], exact, bound, what=f"addmm {M}x{N}x{K}")
+    # batch invariance carries over: row 0 alone gives the same bits
+    C1 = torch.empty(1, N, dtype=torch.float32, device="cuda")
+    bi.addmm(Bv, A[:1], W, C1)
+    assert torch.equal(C1.view(torch.int32), C[:1].view(torch.int32))

@@ -57,6 +57,19 @@ def test_rmsnorm_closed_form():
     assert np.array_equal(rms(ones, w, eps=0.0), np.tile(w, (3, 1)))
 
 
+def test_rmsnorm_product_order_rows():
+    """The rows of the oracle's product-order pin (x = k/16, |k| <= 63, so
+    the sum of squares is exact in any order): some outputs change if the
+    two final products are taken in another order, and the kernel must
+    give the oracle's bits on all of them."""
+    g = np.random.default_rng(2)
+    k = g.integers(-63, 64, size=(512, 4096))
+    x = torch.from_numpy((k / 16.0).astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    w = torch.from_numpy((g.standard_normal(4096) * 0.1 + 1.0).astype(np.float32)).to(torch.bfloat16)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(rms(x, wb), oracle.rmsnorm_canon(x, wb))
+
+
 @pytest.fixture(scope="module")
 def logits():
     return synth.logits_inputs(4096, 151936, seed=0)

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_tol, dev, dev_bf16, host_bits
+from helpers import assert_tol, check_plan_table, dev, dev_bf16, host_bits
 from invariant_bi_lora_b200 import bi, synth
 
 pytestmark = pytest.mark.gpu
@@ -64,6 +64,26 @@ def test_cfg1_replay_100(cfg1):
     exact, bound = oracle.shrink_exact(*cfg1)
     for o in outs_atomic:
         assert_tol(o.view(np.float32), exact, bound, what="atomic replay")
+
+
+def test_atomic_varies_where_tree_does_not(cfg1):
+    """The nondeterminism the split-K study measures ("Reproducible LoRA
+    Inference ...", Highlights): identical-input replays of the atomic
+    split-K shrink give more than one bit pattern, while the tree combine
+    gives one.  Up to 10,000 replays, stopping at the first change."""
+    x, at = (dev_bf16(a) for a in cfg1)
+    first_tree = host_bits(run_shrink(x, at, 8, "tree"))
+    first_atomic = host_bits(run_shrink(x, at, 8, "atomic"))
+    varied = 0
+    for i in range(10000):
+        if not np.array_equal(host_bits(run_shrink(x, at, 8, "atomic")), first_atomic):
+            varied = i + 1
+            break
+        if i % 50 == 0:
+            assert np.array_equal(host_bits(run_shrink(x, at, 8, "tree")), first_tree)
+    assert varied, "10,000 atomic replays all gave the same bits"
+    for _ in range(20):
+        assert np.array_equal(host_bits(run_shrink(x, at, 8, "tree")), first_tree)
 
 
 def test_leaf_tree_bit_exact(cfg1):
@@ -186,9 +206,11 @@ def test_plan_matches_oracle(cfg4):
     assert np.array_equal(perm[:offs[8]], want_perm)
     invalid = np.nonzero((ids < 0) | (ids >= 8))[0]
     assert np.array_equal(perm[offs[8]:], invalid)
+    check_plan_table(plan, np.concatenate([want_perm, invalid]).astype(np.int32), offs, 8)
 
 
-@pytest.mark.parametrize("M,n_ad", [(1, 1), (5, 3), (1000, 8), (4096, 8), (3000, 256), (0, 4)])
+@pytest.mark.parametrize("M,n_ad", [(1, 1), (5, 3), (1000, 8), (4096, 8), (3000, 256), (0, 4),
+                                    (4097, 2), (12289, 8), (65536, 256)])
 def test_plan_shapes(M, n_ad):
     ids = synth.adapter_ids(M, n_ad, seed=M + n_ad)
     plan = bi.lora_plan(dev(ids), n_ad).cpu().numpy() if M else None
@@ -197,6 +219,8 @@ def test_plan_shapes(M, n_ad):
     want_perm, want_offs = oracle.segment(ids, n_ad)
     assert np.array_equal(plan[M:M + n_ad + 1], want_offs)
     assert np.array_equal(plan[:M], want_perm)
+    assert plan[M + n_ad + 1] == M
+    check_plan_table(plan, want_perm, plan[M:M + n_ad + 2], n_ad)
 
 
 @pytest.mark.parametrize("r", [8, 16, 64])
