@@ -64,6 +64,8 @@ def _load():
         "or_gemm_exact": (None, [P, P, L, L, L, P, L, P, P, I]),
         "or_addmm_exact": (None, [P, P, P, L, L, L, P, L, P, P, I]),
         "or_segment": (None, [P, L, I, P, P]),
+        "or_attn_decode_exact": (None, [P, P, P, P, L, L, L, L, L, D, P, I]),
+        "or_attn_decode_canon": (None, [P, P, P, P, L, L, L, L, L, F, P, I]),
         "or_rmsnorm_exact": (None, [P, P, L, L, D, P, I]),
         "or_rmsnorm_canon": (None, [P, P, L, L, F, P, I]),
         "or_rmsnorm_inv_canon": (F, [P, L, F]),
@@ -244,6 +246,37 @@ def addmm_exact(bias, a, w, rows=None, nthreads=None):
     _load().or_addmm_exact(_p(bias), _p(a), _p(w), M, N, K, rp, nr if rows is not None else 0,
                            _p(C), _p(b), _nt(nthreads))
     return C, b
+
+
+def _attn_args(q, k, v, lens):
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    lens = _c(lens, np.int32)
+    B, Hq, D = q.shape
+    B2, Hkv, Lmax, D2 = k.shape
+    assert B2 == B and D2 == D and v.shape == k.shape and lens.shape == (B,) and Hq % Hkv == 0
+    return q, k, v, lens, B, Hq, Hkv, D, Lmax
+
+
+def attn_decode_exact(q, k, v, lens, scale, nthreads=None):
+    """Decode attention in fp64: q bf16 [B,Hq,D]; k, v bf16 [B,Hkv,Lmax,D];
+    lens int32 [B].  Returns out float64 [B,Hq,D]."""
+    q, k, v, lens, B, Hq, Hkv, D, Lmax = _attn_args(q, k, v, lens)
+    out = np.empty((B, Hq, D), np.float64)
+    _load().or_attn_decode_exact(_p(q), _p(k), _p(v), _p(lens), B, Hq, Hkv, D, Lmax, float(scale), _p(out),
+                                 _nt(nthreads))
+    return out
+
+
+def attn_decode_canon(q, k, v, lens, scale, nthreads=None):
+    """Decode attention in the canonical fp32 order (256-key chunk frames,
+    perfect trees, the written exp).  Returns out float32 [B,Hq,D]."""
+    q, k, v, lens, B, Hq, Hkv, D, Lmax = _attn_args(q, k, v, lens)
+    out = np.empty((B, Hq, D), np.float32)
+    _load().or_attn_decode_canon(_p(q), _p(k), _p(v), _p(lens), B, Hq, Hkv, D, Lmax, float(np.float32(scale)),
+                                 _p(out), _nt(nthreads))
+    return out
 
 
 # ------------------------------------------------------------- row ops

@@ -342,6 +342,121 @@ void or_segment(const int32_t *ids, long M, int n_ad, int32_t *perm, int32_t *of
 }
 
 /* ------------------------------------------------------------------ */
+/* Decode attention with a fixed-size KV split ["Restoring AI           */
+/* Reproducibility", 2-3 (attention) and 3-2 (fixed-size split)].       */
+/* One query row per (sequence b, query head h); the kv head is          */
+/* h / (Hq / Hkv).  q bf16 [B][Hq][D]; k, v bf16 [B][Hkv][Lmax][D];     */
+/* lens int32 [B]; out [B][Hq][D].                                       */
+/* ------------------------------------------------------------------ */
+
+/* Exact: out = softmax(scale * q.k_j)_j . v_j over j < lens[b], in
+ * double; a sequence of length 0 gives 0. */
+void or_attn_decode_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *lens,
+                          long B, long Hq, long Hkv, long D, long Lmax, double scale, double *out, int nthreads)
+{
+    #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < B * Hq; bh++) {
+        long b = bh / Hq, h = bh % Hq, hk = h / (Hq / Hkv), L = lens[b];
+        const uint16_t *qr = q + bh * D;
+        const uint16_t *kb = k + (b * Hkv + hk) * Lmax * D;
+        const uint16_t *vb = v + (b * Hkv + hk) * Lmax * D;
+        double *o = out + bh * D;
+        for (long d = 0; d < D; d++) o[d] = 0.0;
+        if (L <= 0) continue;
+        double *s = (double *)malloc(sizeof(double) * (size_t)L);
+        double m = -INFINITY;
+        for (long j = 0; j < L; j++) {
+            double t = 0.0;
+            for (long d = 0; d < D; d++) t += bf(qr[d]) * bf(kb[j * D + d]);
+            s[j] = scale * t;
+            if (s[j] > m) m = s[j];
+        }
+        double den = 0.0;
+        for (long j = 0; j < L; j++) { s[j] = exp(s[j] - m); den += s[j]; }
+        for (long j = 0; j < L; j++)
+            for (long d = 0; d < D; d++) o[d] += s[j] * bf(vb[j * D + d]);
+        for (long d = 0; d < D; d++) o[d] /= den;
+        free(s);
+    }
+}
+
+/* Perfect binary tree over n = 2^k fp32 values (stride apart), pairs
+ * (0,1), (2,3), ... first: the frame sums of the attention below. */
+static float or_frame_tree(float *v, long n)
+{
+    for (long w = 1; w < n; w *= 2)
+        for (long i = 0; i + w < n; i += 2 * w) v[i] = v[i] + v[i + w];
+    return v[0];
+}
+
+/* Canonical fp32 order.  Chunk c holds keys [256c, 256c + 256) as a frame
+ * of 256 slots; slots past the sequence's length hold p = 0 and add +0.
+ *   s_j  = fl(fl(perfect tree over d of q_d * k_jd) * scale)  (the
+ *          products of two bf16 values are exact in fp32; D = 2^k)
+ *   m_c  = max of s_j over the chunk's keys
+ *   p_j  = or_exp(fl(s_j - m_c))
+ *   l_c  = perfect tree over the 256 slots of p_j
+ *   o_cd = perfect tree over the 256 slots of fl(p_j * v_jd)
+ * Combine over the n = ceil(L / 256) chunks, padded to the next power of
+ * two P with zero chunks:
+ *   M = max_c m_c;  a_c = or_exp(fl(m_c - M))
+ *   l = perfect tree over P of fl(a_c * l_c);  O_d = same of fl(a_c * o_cd)
+ *   out_d = fl(O_d / l)
+ * Every order is fixed by the sequence's own length, never by the batch or
+ * by how chunks are shared among workers. */
+void or_attn_decode_canon(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *lens,
+                          long B, long Hq, long Hkv, long D, long Lmax, float scale, float *out, int nthreads)
+{
+    #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < B * Hq; bh++) {
+        long b = bh / Hq, h = bh % Hq, hk = h / (Hq / Hkv), L = lens[b];
+        const uint16_t *qr = q + bh * D;
+        const uint16_t *kb = k + (b * Hkv + hk) * Lmax * D;
+        const uint16_t *vb = v + (b * Hkv + hk) * Lmax * D;
+        float *o = out + bh * D;
+        for (long d = 0; d < D; d++) o[d] = 0.0f;
+        if (L <= 0) continue;
+        long n = (L + 255) / 256, P = 1;
+        while (P < n) P *= 2;
+        float *mc = (float *)calloc((size_t)P, sizeof(float));
+        float *lc = (float *)calloc((size_t)P, sizeof(float));
+        float *oc = (float *)calloc((size_t)(P * D), sizeof(float));
+        float *tmp = (float *)malloc(sizeof(float) * (size_t)(D > 256 ? D : 256));
+        float *pj = (float *)malloc(sizeof(float) * 256);
+        for (long c = 0; c < n; c++) {
+            long j0 = 256 * c, nj = L - j0 < 256 ? L - j0 : 256;
+            float m = -INFINITY;
+            float s[256];
+            for (long i = 0; i < nj; i++) {
+                for (long d = 0; d < D; d++) tmp[d] = or_bf16_to_f32(qr[d]) * or_bf16_to_f32(kb[(j0 + i) * D + d]);
+                s[i] = or_frame_tree(tmp, D) * scale;
+                if (s[i] > m) m = s[i];
+            }
+            mc[c] = m;
+            for (long i = 0; i < 256; i++) pj[i] = i < nj ? or_exp(s[i] - m) : 0.0f;
+            for (long i = 0; i < 256; i++) tmp[i] = pj[i];
+            lc[c] = or_frame_tree(tmp, 256);
+            for (long d = 0; d < D; d++) {
+                for (long i = 0; i < 256; i++) tmp[i] = i < nj ? pj[i] * or_bf16_to_f32(vb[(j0 + i) * D + d]) : 0.0f;
+                oc[c * D + d] = or_frame_tree(tmp, 256);
+            }
+        }
+        float M = mc[0];
+        for (long c = 1; c < n; c++) if (mc[c] > M) M = mc[c];
+        float *ac = (float *)calloc((size_t)P, sizeof(float));
+        for (long c = 0; c < n; c++) ac[c] = or_exp(mc[c] - M);
+        float *col = (float *)malloc(sizeof(float) * (size_t)P);
+        for (long c = 0; c < P; c++) col[c] = ac[c] * lc[c];
+        float l = or_frame_tree(col, P);
+        for (long d = 0; d < D; d++) {
+            for (long c = 0; c < P; c++) col[c] = ac[c] * oc[c * D + d];
+            o[d] = or_frame_tree(col, P) / l;
+        }
+        free(col); free(ac); free(pj); free(tmp); free(oc); free(lc); free(mc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* RMSNorm ["Restoring AI Reproducibility" 2-3, 3-1]                    */
 /* ------------------------------------------------------------------ */
 

@@ -40,6 +40,13 @@ MUTANTS = [
      "yb[j] = (double)y[m * r + j];"),
     ("gemm: W read transposed", "double p = av[k] * bf(wr[k]);", "double p = av[k] * bf(W[k * N + n]);"),
     ("addmm: bias indexed by row", "C[i * N + n] += bf(bias[n]);", "C[i * N + n] += bf(bias[i % N]);"),
+    ("attention: running sum inside a chunk",
+     "oc[c * D + d] = or_frame_tree(tmp, 256);",
+     "{ float acc = 0.0f; for (long i = 0; i < 256; i++) acc = acc + tmp[i]; oc[c * D + d] = acc; }"),
+    ("attention: chunk weights dropped", "for (long c = 0; c < n; c++) ac[c] = or_exp(mc[c] - M);",
+     "for (long c = 0; c < n; c++) ac[c] = 1.0f;"),
+    ("attention exact: softmax without the max shift", "for (long j = 0; j < L; j++) { s[j] = exp(s[j] - m); den += s[j]; }",
+     "for (long j = 0; j < L; j++) { s[j] = exp(s[j]); den += s[j] * (1.0 + 1e-9); }"),
     ("segment: tokens scattered in reverse order",
      "if (ids[t] >= 0 && ids[t] < n_ad) perm[count[ids[t]]++] = (int32_t)t;",
      "if (ids[M - 1 - t] >= 0 && ids[M - 1 - t] < n_ad) perm[count[ids[M - 1 - t]]++] = (int32_t)(M - 1 - t);"),

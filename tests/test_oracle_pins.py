@@ -503,3 +503,85 @@ def test_mean_canon_order(oracle_mod):
     x[0, 0], x[0, 4096], x[0, 4] = 1e8, 1.0, -1e8
     assert oracle_mod.mean_canon(x)[0] == 0.0
     assert oracle_mod.mean_exact(x)[0] == 1.0 / 8192
+
+
+# ------------------------------------------------------- decode attention
+# "Restoring AI Reproducibility", 2-3 (attention) and 3-2 (a fixed-size
+# split of the KV cache, so the order depends on nothing but the sequence).
+
+def _bf(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_attn_exact_vs_torch(oracle_mod):
+    g = np.random.default_rng(21)
+    B, Hq, Hkv, D, Lmax = 3, 4, 2, 64, 300
+    q = _bf(g.standard_normal((B, Hq, D)))
+    k = _bf(g.standard_normal((B, Hkv, Lmax, D)))
+    v = _bf(g.standard_normal((B, Hkv, Lmax, D)))
+    lens = np.array([300, 1, 129], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    got = oracle_mod.attn_decode_exact(q, k, v, lens, scale)
+    qf, kf, vf = (torch.from_numpy(oracle_mod.bf16_to_f32(a).astype(np.float64)) for a in (q, k, v))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            L = int(lens[b])
+            w = torch.softmax(scale * (kf[b, hk, :L] @ qf[b, h]), dim=0)
+            np.testing.assert_allclose(got[b, h], (w @ vf[b, hk, :L]).numpy(), rtol=1e-12, atol=1e-12)
+    # a sequence of length 0 gives 0
+    z = oracle_mod.attn_decode_exact(q, k, v, np.array([0, 5, 0], np.int32), scale)
+    assert np.all(z[0] == 0) and np.all(z[2] == 0)
+
+
+def test_attn_canon_vs_exact(oracle_mod):
+    g = np.random.default_rng(22)
+    B, Hq, Hkv, D, Lmax = 2, 8, 2, 128, 1100
+    q = _bf(g.standard_normal((B, Hq, D)))
+    k = _bf(g.standard_normal((B, Hkv, Lmax, D)))
+    v = _bf(g.standard_normal((B, Hkv, Lmax, D)))
+    lens = np.array([1100, 517], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    c = oracle_mod.attn_decode_canon(q, k, v, lens, scale).astype(np.float64)
+    e = oracle_mod.attn_decode_exact(q, k, v, lens, scale)
+    assert np.max(np.abs(c - e)) <= 1e-5 * np.max(np.abs(e)) + 1e-6
+
+
+def test_attn_canon_closed_forms(oracle_mod):
+    D, Lmax = 128, 1300
+    q = _bf(np.random.default_rng(23).standard_normal((1, 1, D)))
+    zero_k = np.zeros((1, 1, Lmax, D), np.uint16)                  # every score 0, every p = 1
+    # constant value rows: out = that row exactly, at any length
+    vrow = _bf(np.linspace(-3, 3, D))
+    v = np.tile(vrow, (1, 1, Lmax, 1))
+    for L in (1, 5, 255, 256, 257, 1280, 1300):
+        out = oracle_mod.attn_decode_canon(q, zero_k, v, np.array([L], np.int32), 0.125)
+        assert np.array_equal(out[0, 0], oracle_mod.bf16_to_f32(vrow)), L
+    # one dominant key (score > 103 above the rest): out = its value row
+    k = np.zeros((1, 1, Lmax, D), np.uint16)
+    qd = np.zeros((1, 1, D), np.float32)
+    qd[0, 0, 0] = 16.0
+    kd = np.zeros((1, 1, Lmax, D), np.float32)
+    kd[0, 0, 700, 0] = 64.0                                        # score 1024 * 0.125 = 128
+    vals = _bf(np.random.default_rng(24).standard_normal((1, 1, Lmax, D)))
+    out = oracle_mod.attn_decode_canon(_bf(qd), _bf(kd), vals, np.array([1300], np.int32), 0.125)
+    assert np.array_equal(out[0, 0], oracle_mod.bf16_to_f32(vals[0, 0, 700]))
+
+
+def test_attn_canon_frame_order(oracle_mod):
+    """The two frames of the reading.  Inside a chunk, L = 5 keys with p = 1
+    and values [2^24, 0, 1, 1, 0]: the padded 256-slot perfect tree pairs
+    (2^24 + 0) and (1 + 1) and gives 2^24 + 2 exactly (a halving tree over 5
+    or a running sum loses both 1's: 2^24).  Across chunks, 5 full chunks
+    whose sums are [2^24, 0, 1, 1, 0] (values 2^16, 0, 2^-8, 2^-8, 0): the
+    chunk count padded to 8 gives the same pairing.  out = fl((2^24+2)/L)."""
+    D = 32
+    q = np.zeros((1, 1, D), np.uint16)
+    for L, col in ((5, [2.0 ** 24, 0.0, 1.0, 1.0, 0.0]),
+                   (1280, np.repeat([2.0 ** 16, 0.0, 2.0 ** -8, 2.0 ** -8, 0.0], 256))):
+        vf = np.zeros((1, 1, L, D), np.float32)
+        vf[0, 0, :, 0] = col
+        out = oracle_mod.attn_decode_canon(q, np.zeros((1, 1, L, D), np.uint16), _bf(vf), np.array([L], np.int32), 1.0)
+        want = F32(F32(2.0 ** 24 + 2) / F32(L))
+        assert f32bits(out[0, 0, 0]) == f32bits(want), L
+        assert f32bits(want) != f32bits(F32(F32(2.0 ** 24) / F32(L)))
