@@ -7,9 +7,12 @@ shaped like the pages' workloads:
   shrink    segmented LoRA shrink, M=4096, K=4096, r=16, split-K 8:
             tree (deterministic), atomic, unsplit
   expand    segmented LoRA expand r=16 -> N=4096
+  fused     shrink (tree, split-K 8) and expand in one launch, y on chip
   shrink16  LoRA shrink M=16, K=4096, r=16: tree s=8, atomic s=8, unsplit
   gemm      batch-invariant GEMM M=4096, N=4096, K=4096 (tcgen05)
   treegemm  TP-invariant tree GEMM M=2048, N=4096, K=16384, 8 emulated shards
+  attn      decode attention, fixed-size KV split: 32 sequences x 2048 tokens,
+            32 query heads over 8 kv heads, head size 128
   rmsnorm   4096 x 4096 bf16
   lsm       log_softmax 4096 x 151936 fp32
   mean      mean of the same 4096 x 151936 fp32 rows
@@ -57,6 +60,22 @@ def shrink_bytes(M=M4, K=K4, r=R4, n_ad=NAD):
 def expand_bytes(M=M4, N=4096, r=R4, n_ad=NAD):
     """y, every adapter's B, the fp32 out write and the token ids."""
     return M * r * 4 + n_ad * N * r * 2 + M * N * 4 + 4 * M
+
+
+def fused_bytes(M=M4, K=K4, N=4096, r=R4, n_ad=NAD):
+    """Fused shrink + expand: x, every adapter's A and B, the fp32 out
+    write, the plan's token ids and tile headers (y never leaves the chip)."""
+    return M * K * 2 + n_ad * r * K * 2 + n_ad * N * r * 2 + M * N * 4 + 4 * M + 16 * ((M + 63) // 64 + n_ad + 1)
+
+
+# decode attention: 32 sequences of 2048 cached tokens, 32 query heads over
+# 8 kv heads, head size 128 (a grouped-query decoder layer)
+ATT_B, ATT_HQ, ATT_HKV, ATT_D, ATT_L = 32, 32, 8, 128, 2048
+
+
+def attn_bytes(B, Hq, Hkv, D, lens):
+    """K and V of every sequence's cached tokens, q, and the fp32 out."""
+    return sum(lens) * Hkv * D * 2 * 2 + B * Hq * D * 2 + B * Hq * D * 4
 
 
 SHRINK_BYTES = shrink_bytes()
@@ -184,6 +203,14 @@ class Workload:
         self.logits = torch.from_numpy(synth.logits_inputs(4096, 151936, seed=seed)).cuda()
         self.lsm = torch.empty_like(self.logits)
         self.mean = torch.empty(4096, dtype=torch.float32, device="cuda")
+        g = np.random.default_rng(seed)
+        self.aq = torch.randn(ATT_B, ATT_HQ, ATT_D, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16).cuda()
+        self.ak = torch.randn(ATT_B, ATT_HKV, ATT_L, ATT_D, generator=torch.Generator().manual_seed(seed + 1)).to(torch.bfloat16).cuda()
+        self.av = torch.randn(ATT_B, ATT_HKV, ATT_L, ATT_D, generator=torch.Generator().manual_seed(seed + 2)).to(torch.bfloat16).cuda()
+        self.alens = torch.full((ATT_B,), ATT_L, dtype=torch.int32, device="cuda")
+        self.aout = torch.empty(ATT_B, ATT_HQ, ATT_D, dtype=torch.float32, device="cuda")
+        self.aws = torch.empty(bi.attn_decode_ws_bytes(ATT_B, ATT_HQ, ATT_D, ATT_L), dtype=torch.uint8, device="cuda")
+        del g
         self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
         self.flush_f = self.flush.view(torch.float32)
         self.flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
@@ -204,12 +231,16 @@ class Workload:
              SHRINK_BYTES, 2 * M4 * K4 * R4, "hbm", 1),
             ("expand", lambda: bi.lora_expand_segmented(self.y, self.B, self.plan, self.out),
              expand_bytes(), 2 * M4 * 4096 * R4, "hbm", 1),
+            ("fused_shrink_expand", lambda: bi.lora_fused(self.x, self.A, self.B, self.plan, self.out, splits=8),
+             fused_bytes(), 2 * M4 * K4 * R4 + 2 * M4 * 4096 * R4, "hbm", 1),
             ("shrink16_tree_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "tree"),
              16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
             ("shrink16_atomic_s8", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 8, "atomic"),
              16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
             ("shrink16_unsplit", lambda: bi.lora_shrink(self.x16, self.A16, self.y16, 1, "unsplit"),
              16 * 4096 * 2 * 2 + 16 * 16 * 4, 2 * 16 * 4096 * 16, "hbm", 1),
+            ("attn_decode", lambda: bi.attn_decode(self.aq, self.ak, self.av, self.alens, self.aout, ws=self.aws),
+             attn_bytes(ATT_B, ATT_HQ, ATT_HKV, ATT_D, [ATT_L] * ATT_B), 4 * ATT_B * ATT_HQ * ATT_L * ATT_D, "hbm", 2),
             ("rmsnorm", lambda: bi.rmsnorm(self.xr, self.wr, self.yr, 1e-6),
              4096 * 4096 * 4 + 4096 * 2, 0, "hbm", 1),
             ("log_softmax", lambda: bi.log_softmax(self.logits, self.lsm), lsm_bytes, 0, "hbm", 1),
@@ -488,6 +519,20 @@ class Sweep:
             self.add("d4", f"expand r={r}", {"M": M4, "N": 4096, "r": r, "adapters": NAD}, "hbm",
                      expand_bytes(r=r), 2 * M4 * 4096 * r,
                      lambda y=y, B=B, plan=plan: bi.lora_expand_segmented(y, B, plan, wl.out))
+            self.add("N4", f"fused shrink+expand s=8 r={r}", {"M": M4, "K": K4, "N": 4096, "r": r, "adapters": NAD},
+                     "hbm", fused_bytes(r=r), 2 * M4 * K4 * r + 2 * M4 * 4096 * r,
+                     lambda X=X, A=A, B=B, plan=plan: bi.lora_fused(X, A, B, plan, wl.out, splits=8))
+        gen = torch.Generator().manual_seed(7)
+        for Bq, L in ((1, 256), (1, 4096), (8, 16384), (32, 1024), (64, 4096)):
+            q = torch.randn(Bq, 32, 128, generator=gen).to(torch.bfloat16).cuda()
+            kk = torch.randn(Bq, 8, L, 128, generator=gen).to(torch.bfloat16).cuda()
+            vv = torch.randn(Bq, 8, L, 128, generator=gen).to(torch.bfloat16).cuda()
+            lens = torch.full((Bq,), L, dtype=torch.int32, device="cuda")
+            out = torch.empty(Bq, 32, 128, dtype=torch.float32, device="cuda")
+            ws = torch.empty(bi.attn_decode_ws_bytes(Bq, 32, 128, L), dtype=torch.uint8, device="cuda")
+            self.add("N1", f"attn_decode B={Bq} L={L}", {"B": Bq, "Hq": 32, "Hkv": 8, "D": 128, "L": L}, "hbm",
+                     attn_bytes(Bq, 32, 8, 128, [L] * Bq), 4 * Bq * 32 * L * 128,
+                     lambda q=q, kk=kk, vv=vv, lens=lens, out=out, ws=ws: bi.attn_decode(q, kk, vv, lens, out, ws=ws))
         a, w = synth.gemm_inputs(2048, 4096, 16384, seed=1)
         self.ta, self.tw = dev_bf16(a), dev_bf16(w)
         self.tc = torch.empty(2048, 4096, dtype=torch.float32, device="cuda")

@@ -146,6 +146,19 @@ bi_status bi_lora_shrink_segmented_noalloc(const void *x, const void *A, const i
                                            int n_adapters, float *y, int M, int K, int r,
                                            int splits, int mode, bi_stream_t stream);
 
+/* Fused segmented LoRA [LoRA Q&A: the two low-rank products]: the      */
+/* segmented shrink (split-K `splits` in mode TREE, or UNSPLIT when      */
+/* splits = 1) and then out[t] (+)= bf16(y[t]) . B_{id[t]}^T, in one     */
+/* launch.  y stays on chip (the CTAs of a row tile share it through     */
+/* distributed shared memory); it is also written to y when y != NULL.   */
+/* Bitwise the same as bi_lora_shrink_segmented followed by              */
+/* bi_lora_expand_segmented.  B bf16 [n_adapters][N][r]; out fp32 [M][N] */
+/* (16-byte aligned); N % 8 == 0; plan from bi_lora_plan; other          */
+/* requirements as those two calls.  Mode ATOMIC has no fused form.      */
+bi_status bi_lora_fused(const void *x, const void *A, const void *B, const void *plan,
+                        int n_adapters, float *y, float *out, int M, int K, int r, int N,
+                        int splits, int accumulate, bi_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* LoRA expand [LoRA Q&A: the second low-rank product]:                 */
 /*   e[t][n] = sum_j bf16(y[t][j]) * B[n][j]                            */
@@ -250,6 +263,31 @@ bi_status bi_mean(const float *x, float *out, int rows, int n, bi_stream_t strea
  * shortcut on packed two-lane fp32 instructions (elements 2k and 2k+1 form
  * one pair).  Other values of which: BI_ERR_INVALID_ARG. */
 bi_status bi_math_spec(const float *x, float *y, size_t n, int which, bi_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* Batch-invariant decode attention with a fixed-size KV split          */
+/* ["Restoring AI Reproducibility", 2-3 and 3-2].  One query row per    */
+/* (sequence b, query head h) attends to keys [0, lens[b]) of kv head   */
+/* h / (Hq / Hkv):  out = softmax(scale * q . k_j) . v_j.  The keys are */
+/* cut into chunks of 256 slots whatever the batch; every sum is a      */
+/* perfect tree (the dot product over D; the 256 slots of a chunk, zero */
+/* past the length; the chunks, padded to a power of two), exp is       */
+/* bi_math_spec's, so row (b, h) is bitwise the same for any batch,     */
+/* position, Lmax or number of CTAs.  The exact order:                  */
+/*   s_j = fl(fl(tree_d q_d k_jd) * scale); m_c = chunk max;            */
+/*   p_j = exp(fl(s_j - m_c)); l_c = tree p_j; o_cd = tree fl(p_j v_jd);*/
+/*   M = max m_c; a_c = exp(fl(m_c - M)); l = tree fl(a_c l_c);         */
+/*   O_d = tree fl(a_c o_cd); out_d = fl(O_d / l); lens[b] = 0 gives 0. */
+/* q bf16 [B][Hq][D]; k, v bf16 [B][Hkv][Lmax][D]; lens int32 [B] with  */
+/* 0 <= lens[b] <= Lmax (longer lengths are cut at Lmax); out fp32      */
+/* [B][Hq][D].  D in {64, 128, 256}; Hq / Hkv in {1, 2, 4, 8}; q, k, v, */
+/* out 16-byte aligned.  ws: bi_attn_decode_ws_bytes(B, Hq, D, Lmax)    */
+/* bytes of caller memory for the chunk partials.                       */
+/* ------------------------------------------------------------------ */
+size_t bi_attn_decode_ws_bytes(int B, int Hq, int D, int Lmax);
+bi_status bi_attn_decode(const void *q, const void *k, const void *v, const int32_t *lens,
+                         float *out, int B, int Hq, int Hkv, int D, int Lmax, float scale,
+                         void *ws, size_t ws_bytes, bi_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* Status                                                               */

@@ -39,6 +39,7 @@ _SIGS = {
     "bi_lora_plan": (I, [P, I, I, P, Z, P]),
     "bi_lora_shrink_segmented": (I, [P, P, P, I, P, I, I, I, I, I, P]),
     "bi_lora_shrink_segmented_noalloc": (I, [P, P, P, I, P, I, I, I, I, I, P]),
+    "bi_lora_fused": (I, [P, P, P, P, I, P, P, I, I, I, I, I, I, P]),
     "bi_lora_expand": (I, [P, P, P, I, I, I, I, P]),
     "bi_lora_expand_segmented": (I, [P, P, P, I, P, I, I, I, I, P]),
     "bi_gemm": (I, [P, P, P, I, I, I, I, P]),
@@ -51,6 +52,8 @@ _SIGS = {
     "bi_log_softmax": (I, [P, P, I, I, P]),
     "bi_mean": (I, [P, P, I, I, P]),
     "bi_math_spec": (I, [P, P, Z, I, P]),
+    "bi_attn_decode_ws_bytes": (Z, [I, I, I, I]),
+    "bi_attn_decode": (I, [P, P, P, P, P, I, I, I, I, I, F, P, Z, P]),
     "bi_get_device_status": (I, [P]),
     "bi_status_string": (ctypes.c_char_p, [I]),
     "bi_selftest_bounded_wait": (I, [I, P]),
@@ -171,6 +174,32 @@ def lora_shrink_segmented_noalloc(x, A, ids, y, splits=8, mode="tree", stream=No
     _call("bi_lora_shrink_segmented_noalloc", _ptr(x), _ptr(A), _ptr(ids), n_ad, _ptr(y), M, K, r,
           splits, MODES[mode], _stream(stream))
     return y
+
+
+def lora_fused(x, A, B, plan, out, y=None, splits=8, accumulate=False, stream=None):
+    """Segmented shrink then expand in one launch: out[t] (+)= bf16(y[t]) .
+    B_{id[t]}^T with y = x[t] . A_{id[t]} (split-K tree, or unsplit when
+    splits = 1); y is also written when given.  A bf16 [n_ad, r, K],
+    B bf16 [n_ad, N, r], out fp32 [M, N]."""
+    _check(x, "x", torch.bfloat16, 2)
+    _check(A, "A", torch.bfloat16, 3)
+    _check(B, "B", torch.bfloat16, 3)
+    _check(plan, "plan", torch.int32, 1)
+    _check(out, "out", torch.float32, 2)
+    M, K = x.shape
+    n_ad, r, K2 = A.shape
+    N = B.shape[1]
+    if K2 != K or tuple(B.shape) != (n_ad, N, r) or tuple(out.shape) != (M, N):
+        raise ValueError("shape mismatch")
+    if y is not None:
+        _check(y, "y", torch.float32, 2)
+        if tuple(y.shape) != (M, r):
+            raise ValueError("shape mismatch")
+    if plan.numel() * 4 < lora_plan_bytes(M, n_ad):
+        raise ValueError("plan too small")
+    _call("bi_lora_fused", _ptr(x), _ptr(A), _ptr(B), _ptr(plan), n_ad, _ptr(y), _ptr(out), M, K, r, N,
+          splits, int(bool(accumulate)), _stream(stream))
+    return out
 
 
 def lora_expand(y, B, out, accumulate=False, stream=None):
@@ -322,6 +351,34 @@ def math_spec(x, y, which, stream=None):
     _call("bi_math_spec", _ptr(x), _ptr(y), x.numel(), {"exp": 0, "log": 1, "exp_fast": 2, "exp_fast2": 3}[which],
           _stream(stream))
     return y
+
+
+# ------------------------------------------------------------- attention
+
+def attn_decode_ws_bytes(B, Hq, D, Lmax):
+    return int(lib().bi_attn_decode_ws_bytes(B, Hq, D, Lmax))
+
+
+def attn_decode(q, k, v, lens, out, scale=None, ws=None, stream=None):
+    """Decode attention with a fixed-size KV split: q bf16 [B, Hq, D];
+    k, v bf16 [B, Hkv, Lmax, D]; lens int32 [B]; out fp32 [B, Hq, D]."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(lens, "lens", torch.int32, 1)
+    _check(out, "out", torch.float32, 3)
+    B, Hq, D = q.shape
+    B2, Hkv, Lmax, D2 = k.shape
+    if B2 != B or D2 != D or v.shape != k.shape or lens.shape[0] != B or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    need = attn_decode_ws_bytes(B, Hq, D, Lmax)
+    if ws is None:
+        ws = torch.empty(max(need, 4), dtype=torch.uint8, device=q.device)
+    _call("bi_attn_decode", _ptr(q), _ptr(k), _ptr(v), _ptr(lens), _ptr(out), B, Hq, Hkv, D, Lmax, float(scale),
+          _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return out
 
 
 # ------------------------------------------------------------------ status

@@ -78,6 +78,12 @@ struct ShrinkParams {
   int sub;                  // CTA tiles per 64-row table record (64 / bm)
   int rowbytes;             // bytes of one row's K range in one split (lc * 128)
   int x_off, part_off;      // shared-memory offsets of the x rows and the group values
+  // fused expand (register-ring kernel only)
+  int fuse;                 // 1: after y, out (+)= bf16(y) . B^T for the tile
+  const uint16_t *bt;       // [n_ad][N][r] bf16
+  float *out;               // [M][N] fp32
+  int N, accumulate;
+  int yfull_rel, stage_rel; // bytes from `part` to the full y tile, and from it to the strip buffers
   uint8_t merges[kMaxGroupLeaves];   // post-order merges after each leaf
 };
 
@@ -187,14 +193,114 @@ BI_DEV void tile_record(const ShrinkParams &p, int bm, int tile, int lane, int32
   }
 }
 
+// Fused expand ("Reproducible LoRA Inference ...", Q&A: LoRA is a shrink
+// followed by an expand; here y stays on chip).  yfull [bm][r] holds the
+// tile's final y rows in this CTA's shared memory.  Rank q of the S CTAs of
+// the tile computes the 64-column strips j = q, q + S, ... of
+// out[row][n] (+)= sum_j bf16(y[row][j]) * B[adapter][n][j]: per 16-row
+// m-tile and 8-column n-tile one chain of KS = ceil(r/16) MMAs from zero,
+// the same fragments and order as the expand kernel, so the bits equal a
+// separate shrink then expand.  Each warp stages its 16 x 64 strip in
+// shared memory (stride 68 floats) and writes whole 256-byte row segments.
+template <int KS>
+BI_DEV void fused_expand_ks(const ShrinkParams &p, const float *yfull, const int32_t *s_rows, int rows, int adapter,
+                            int q, int S) {
+  float *stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(const_cast<float *>(yfull)) + p.stage_rel);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  const int half = lane >> 4, q4 = (lane & 15) * 4;
+  float(*so)[68] = reinterpret_cast<float(*)[68]>(stage + (size_t)warp * 16 * 68);
+  const int mts = (rows + 15) >> 4;
+  const int strips = (p.N + 63) >> 6;
+  const int my_strips = strips > q ? (strips - q + S - 1) / S : 0;
+  const uint16_t *bad = p.bt + (size_t)adapter * p.N * p.r;
+  for (int combo = warp; combo < mts * my_strips; combo += nwarps) {
+    const int mt = combo % mts, sj = q + S * (combo / mts);
+    const int lr0 = mt * 16 + g, lr1 = lr0 + 8;
+    uint32_t afr[KS][4];
+#pragma unroll
+    for (int st = 0; st < KS; st++) {
+      const int k0 = 16 * st + 2 * c, k1 = k0 + 8;
+      float2 a00 = make_float2(0.f, 0.f), a10 = a00, a01 = a00, a11 = a00;
+      if (k0 < p.r) {
+        a00 = *reinterpret_cast<const float2 *>(yfull + lr0 * p.r + k0);
+        a10 = *reinterpret_cast<const float2 *>(yfull + lr1 * p.r + k0);
+      }
+      if (k1 < p.r) {
+        a01 = *reinterpret_cast<const float2 *>(yfull + lr0 * p.r + k1);
+        a11 = *reinterpret_cast<const float2 *>(yfull + lr1 * p.r + k1);
+      }
+      afr[st][0] = pack_bf16x2(a00.x, a00.y);
+      afr[st][1] = pack_bf16x2(a10.x, a10.y);
+      afr[st][2] = pack_bf16x2(a01.x, a01.y);
+      afr[st][3] = pack_bf16x2(a11.x, a11.y);
+    }
+    const int nbase = sj * 64;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const int n0 = nbase + i * 8;
+      const uint16_t *brow = bad + (size_t)(n0 + g) * p.r;
+      const bool ok = n0 < p.N;
+      uint32_t bfr[KS][2];
+#pragma unroll
+      for (int st = 0; st < KS; st++) {
+        const int k0 = 16 * st + 2 * c, k1 = k0 + 8;
+        bfr[st][0] = ok && k0 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k0)) : 0u;
+        bfr[st][1] = ok && k1 < p.r ? __ldg(reinterpret_cast<const unsigned int *>(brow + k1)) : 0u;
+      }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int st = 0; st < KS; st++) mma_bf16_16816(acc, afr[st], bfr[st], acc);
+      *reinterpret_cast<float2 *>(&so[g][i * 8 + 2 * c]) = make_float2(acc[0], acc[1]);
+      *reinterpret_cast<float2 *>(&so[g + 8][i * 8 + 2 * c]) = make_float2(acc[2], acc[3]);
+    }
+    __syncwarp();
+    const int n = nbase + q4;
+#pragma unroll 2
+    for (int j = 0; j < 8; j++) {
+      const int lr = 2 * j + half, tr = mt * 16 + lr;
+      if (tr < rows && n < p.N) {
+        float4 v = *reinterpret_cast<const float4 *>(&so[lr][q4]);
+        float4 *o = reinterpret_cast<float4 *>(p.out + (size_t)s_rows[tr] * p.N + n);
+        if (p.accumulate) {
+          const float4 old = *o;
+          v.x = __fadd_rn(old.x, v.x);
+          v.y = __fadd_rn(old.y, v.y);
+          v.z = __fadd_rn(old.z, v.z);
+          v.w = __fadd_rn(old.w, v.w);
+        }
+        __stcs(o, v);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+BI_DEV void fused_expand(const ShrinkParams &p, const float *yfull, const int32_t *s_rows, int rows, int adapter, int q,
+                         int S) {
+  switch ((p.r + 15) >> 4) {
+    case 1: fused_expand_ks<1>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 2: fused_expand_ks<2>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 3: fused_expand_ks<3>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 4: fused_expand_ks<4>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 5: fused_expand_ks<5>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 6: fused_expand_ks<6>(p, yfull, s_rows, rows, adapter, q, S); break;
+    case 7: fused_expand_ks<7>(p, yfull, s_rows, rows, adapter, q, S); break;
+    default: fused_expand_ks<8>(p, yfull, s_rows, rows, adapter, q, S); break;
+  }
+}
+
 // The G group values of a row tile (part [G][bm][r], in shared memory,
 // written and visible to the CTA) -> the tile's y rows: the perfect tree over
 // the groups, then the cross-split combine of the mode.  Every thread of the
 // CTA calls it.  In mode TREE with splits > 1 each CTA has made a relaxed
 // cluster arrive on entry; the matching wait comes before the first write
 // into a peer's shared memory.  slots: the exchange slots (mode TREE).
+// With p.fuse, the final y values also go to yfull in every CTA of the tile
+// (all-gather through distributed shared memory), and the tile's expand
+// follows; y itself is written only when p.y is set.
 BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const int32_t *s_rows,
-                        int rows, int bm, int split) {
+                        int rows, int bm, int split, int adapter) {
   const int E = bm * p.r;
   const int r_sh = (p.r & (p.r - 1)) == 0 ? __ffs(p.r) - 1 : -1;
   auto e_row = [&](int e) { return r_sh >= 0 ? e >> r_sh : e / p.r; };
@@ -209,13 +315,21 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
 
   auto out_index = [&](int e) -> size_t { return (size_t)s_rows[e_row(e)] * p.r + e_col(e); };
   const int valid_E = rows * p.r;
+  float *yfull = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(part) + p.yfull_rel);
 
   if (p.mode == BI_SHRINK_ATOMIC) {
     for (int e = threadIdx.x; e < valid_E; e += blockDim.x) atomicAdd(p.y + out_index(e), part[e]);
     return;
   }
   if (p.splits == 1) {
-    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) p.y[out_index(e)] = part[e];
+    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
+      if (p.y) p.y[out_index(e)] = part[e];
+      if (p.fuse) yfull[e] = part[e];
+    }
+    if (p.fuse) {
+      __syncthreads();
+      fused_expand(p, yfull, s_rows, rows, adapter, 0, 1);
+    }
     return;
   }
 
@@ -233,6 +347,12 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
   // the relaxed arrive each CTA made on entry: once this wait returns,
   // every CTA of the cluster is running, so its shared memory may be written
   cluster_wait();
+  // a final y value: to global memory and, fused, to every rank's yfull
+  auto emit = [&](int e, float v) {
+    if (p.y) p.y[out_index(e)] = v;
+    if (p.fuse)
+      for (int t = 0; t < S; t++) cluster.map_shared_rank(yfull, t)[e] = v;
+  };
   if (p.gather0) {
     // small tiles: ranks 1..S-1 push their whole partial into rank 0's
     // slots [S-1][E]; after the barrier rank 0 alone adds and writes y
@@ -244,44 +364,50 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
     }
     cluster_arrive_release();
     cluster_wait_acquire();
-    if (split != 0) return;
-    for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
-      float v[kMaxSplits];
-      v[0] = part[e];
+    if (split == 0) {
+      for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
+        float v[kMaxSplits];
+        v[0] = part[e];
 #pragma unroll
-      for (int q = 1; q < kMaxSplits; q++) v[q] = q < S ? gslots[(size_t)(q - 1) * E + e] : 0.0f;
+        for (int q = 1; q < kMaxSplits; q++) v[q] = q < S ? gslots[(size_t)(q - 1) * E + e] : 0.0f;
+#pragma unroll
+        for (int st = 1; st < kMaxSplits; st <<= 1)
+#pragma unroll
+          for (int q = 0; q + st < kMaxSplits; q += 2 * st)
+            if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
+        emit(e, v[0]);
+      }
+    }
+  } else {
+    const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
+    for (int t = 0; t < S; t++) {
+      if (t == split) continue;
+      float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
+      const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
+      for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
+    }
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    for (int i = threadIdx.x; i < share; i += blockDim.x) {
+      const int e = split * share + i;
+      if (e >= valid_E) break;
+      float v[kMaxSplits];
+#pragma unroll
+      for (int q = 0; q < kMaxSplits; q++)
+        v[q] = q < S ? (q == split ? part[e] : slots[(size_t)q * share + i]) : 0.0f;
 #pragma unroll
       for (int st = 1; st < kMaxSplits; st <<= 1)
 #pragma unroll
         for (int q = 0; q + st < kMaxSplits; q += 2 * st)
           if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
-      p.y[out_index(e)] = v[0];
+      emit(e, v[0]);
     }
-    return;
   }
-  const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
-  for (int t = 0; t < S; t++) {
-    if (t == split) continue;
-    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
-    const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
-    for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
-  }
+  if (!p.fuse) return;
+  // every rank's yfull is complete once all ranks have emitted their shares
   cluster_arrive_release();
   cluster_wait_acquire();
-  for (int i = threadIdx.x; i < share; i += blockDim.x) {
-    const int e = split * share + i;
-    if (e >= valid_E) break;
-    float v[kMaxSplits];
-#pragma unroll
-    for (int q = 0; q < kMaxSplits; q++)
-      v[q] = q < S ? (q == split ? part[e] : slots[(size_t)q * share + i]) : 0.0f;
-#pragma unroll
-    for (int st = 1; st < kMaxSplits; st <<= 1)
-#pragma unroll
-      for (int q = 0; q + st < kMaxSplits; q += 2 * st)
-        if (q + st < S) v[q] = __fadd_rn(v[q], v[q + st]);
-    p.y[out_index(e)] = v[0];
-  }
+  fused_expand(p, yfull, s_rows, rows, adapter, split, S);
 }
 
 // PF: leaves of x in flight per thread, in a register ring.  LG: leaves per
@@ -323,9 +449,16 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   auto e_col = [&](int e) { return r_sh >= 0 ? e & (p.r - 1) : e % p.r; };
 
   if (ti.adapter == p.n_ad) {                       // tokens without an adapter
-    if (p.mode != BI_SHRINK_ATOMIC && split == 0)
+    if (p.mode != BI_SHRINK_ATOMIC && split == 0 && p.y)
       for (int e = threadIdx.x; e < ti.rows * p.r; e += blockDim.x)
         p.y[(size_t)s_rows[e_row(e)] * p.r + e_col(e)] = 0.0f;
+    if (p.fuse && !p.accumulate) {
+      // their expand rows are zero; the splits share the columns
+      const int n4 = p.N >> 2;
+      for (int i = threadIdx.x + split * blockDim.x; i < ti.rows * n4; i += blockDim.x * p.splits)
+        __stcs(reinterpret_cast<float4 *>(p.out + (size_t)s_rows[i / n4] * p.N) + i % n4,
+               make_float4(0.f, 0.f, 0.f, 0.f));
+    }
     if (clustered) cluster_wait();
     return;
   }
@@ -512,7 +645,7 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   }
   __syncthreads();
   float *slots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);
-  finish_tile(p, part, slots, s_rows, ti.rows, bm, split);
+  finish_tile(p, part, slots, s_rows, ti.rows, bm, split, ti.adapter);
 }
 
 // ----------------------------------------------------------------------
@@ -697,7 +830,7 @@ shrink_bulk_kernel(const __grid_constant__ ShrinkParams p) {
   }
   __syncthreads();
   float *slots = reinterpret_cast<float *>(smem + p.g_offset);
-  finish_tile(p, part, slots, s_rows, rows, bm, split);
+  finish_tile(p, part, slots, s_rows, rows, bm, split, adapter);
 }
 
 // ----------------------------------------------------------------------
@@ -852,15 +985,23 @@ static bool bulk_tiling(ShrinkParams &p, int M, bool segmented, int &threads, in
   return smem <= 200 * 1024;
 }
 
+// The expand half of a fused call.
+struct FuseArgs {
+  const void *B;            // [n_ad][N][r] bf16
+  float *out;               // [M][N] fp32
+  int N, accumulate;
+};
+
 // Validates, picks the kernel and its (bit-neutral) tiling and launches.
-// perm / offsets / table are null for the single-adapter call.
+// perm / offsets / table are null for the single-adapter call; fuse is
+// null except for bi_lora_fused.
 bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const int32_t *offsets,
                         const int32_t *table, int n_ad, float *y, int M, int K, int r, int splits, int mode,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const FuseArgs *fuse = nullptr) {
   if (M < 0 || K <= 0 || r <= 0 || n_ad < 1) return BI_ERR_INVALID_ARG;
   if (mode != BI_SHRINK_UNSPLIT && mode != BI_SHRINK_ATOMIC && mode != BI_SHRINK_TREE)
     return BI_ERR_INVALID_ARG;
-  if (M > 0 && (!x || !A || !y)) return BI_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !A || (!y && !fuse))) return BI_ERR_INVALID_ARG;
   if (K % kLeaf != 0 || r % 8 != 0 || r > 128) return BI_ERR_UNSUPPORTED_SHAPE;
   const int L = K / kLeaf;
   if (mode == BI_SHRINK_UNSPLIT && splits != 1) return BI_ERR_UNSUPPORTED_SHAPE;
@@ -885,7 +1026,17 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   p.ngroups = r / ngw;
   if (p.ngroups > 8) return BI_ERR_UNSUPPORTED_SHAPE;
 
-  {
+  if (fuse) {
+    if (mode == BI_SHRINK_ATOMIC) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (fuse->N <= 0 || !fuse->B || !fuse->out) return BI_ERR_INVALID_ARG;
+    if (fuse->N % 8 != 0 || !bi_aligned16(fuse->B) || !bi_aligned16(fuse->out)) return BI_ERR_UNSUPPORTED_SHAPE;
+    p.fuse = 1;
+    p.bt = static_cast<const uint16_t *>(fuse->B);
+    p.out = fuse->out;
+    p.N = fuse->N;
+    p.accumulate = fuse->accumulate ? 1 : 0;
+  }
+  if (!fuse) {
     ShrinkParams q = p;
     int threads = 0, tiles = 0;
     size_t smem = 0;
@@ -938,7 +1089,15 @@ bi_status shrink_launch(const void *x, const void *A, const int32_t *perm, const
   const size_t slot_bytes = mode == BI_SHRINK_TREE && splits > 1 ? (p.gather0 ? (size_t)(splits - 1) * part1 : part1) : 0;
   const size_t base_smem = part_bytes + (p.a_staged ? a_bytes : 0);
   p.g_offset = (int)base_smem;
-  const size_t smem = base_smem + slot_bytes;
+  size_t smem = base_smem + slot_bytes;
+  if (p.fuse) {
+    // the tile's full y rows, then one 16 x 68 float strip buffer per warp
+    smem = (smem + 15) & ~size_t(15);
+    p.yfull_rel = (int)smem;                       // part sits at offset 0
+    const size_t yfull_bytes = ((size_t)bm * r * sizeof(float) + 15) & ~size_t(15);
+    p.stage_rel = (int)yfull_bytes;
+    smem += yfull_bytes + (size_t)warps * 16 * 68 * sizeof(float);
+  }
   p.sub = kPlanTile / bm;
   const int tiles = table ? (int)plan_tiles(M, n_ad) * p.sub : (M + bm - 1) / bm;
 
@@ -972,6 +1131,20 @@ extern "C" bi_status bi_lora_shrink(const void *x, const void *A, float *y, int 
                                     int splits, int mode, bi_stream_t stream) {
   return bi::shrink_launch(x, A, nullptr, nullptr, nullptr, 1, y, M, K, r, splits, mode,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" bi_status bi_lora_fused(const void *x, const void *A, const void *B, const void *plan, int n_adapters,
+                                   float *y, float *out, int M, int K, int r, int N, int splits, int accumulate,
+                                   bi_stream_t stream) {
+  if (M > 0 && !plan) return BI_ERR_INVALID_ARG;
+  if (n_adapters < 1 || n_adapters > bi::kMaxAdapters) return BI_ERR_INVALID_ARG;
+  if (M > 0 && !bi_aligned16(plan)) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (y && !bi_aligned16(y)) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int32_t *perm = static_cast<const int32_t *>(plan);
+  const int32_t *table = perm + bi::plan_table_word(M, n_adapters);
+  bi::FuseArgs f{B, out, N, accumulate};
+  return bi::shrink_launch(x, A, perm, perm + M, table, n_adapters, y, M, K, r, splits,
+                           splits > 1 ? BI_SHRINK_TREE : BI_SHRINK_UNSPLIT, reinterpret_cast<cudaStream_t>(stream), &f);
 }
 
 extern "C" bi_status bi_lora_shrink_segmented(const void *x, const void *A, const void *plan,
