@@ -67,13 +67,15 @@ BI_DEV float counter_fold(int i, float x, float (&lv)[LEVELS > 0 ? LEVELS : 1]) 
 template <int D, int G>
 __global__ void __launch_bounds__(kAttnThreads, 2)
 attn_chunk_kernel(const __grid_constant__ AttnParams p) {
-  constexpr int QT = kAttnThreads / D;              // threads per output column
+  constexpr int QT = 2 * kAttnThreads / D;          // threads per output column pair
   constexpr int SLOTS = kAttnChunk / QT;            // slots per thread in the PV sum
-  constexpr int LV = SLOTS >= 256 ? 8 : SLOTS >= 128 ? 7 : 6;
+  constexpr int LV = SLOTS >= 128 ? 7 : SLOTS >= 64 ? 6 : 5;
+  constexpr int GP = G >= 4 ? G : 4;                // p row padded to a float4
   extern __shared__ __align__(128) uint8_t attn_smem[];
   uint16_t *s_v = reinterpret_cast<uint16_t *>(attn_smem);            // [256][D] bf16
   __shared__ float s_q[G][D];
-  __shared__ float s_p[G][kAttnChunk];
+  __shared__ float s_p[G][kAttnChunk];             // scores
+  __shared__ __align__(16) float s_pt[kAttnChunk][GP];   // p, [slot][head]
   __shared__ float s_red[G][8];
   __shared__ float s_half[G][QT][D];
   __shared__ __align__(8) uint64_t s_bar;
@@ -174,7 +176,7 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
 #pragma unroll
   for (int i = 0; i < G; i++) {
     pv[i] = tid < nj ? bi_exp(__fsub_rn(s_p[i][tid], m_i[i])) : 0.0f;
-    s_p[i][tid] = pv[i];
+    s_pt[tid][i] = pv[i];
     const float lw = warp_tree_sum(pv[i]);
     if (lane == 0) s_red[i][warp] = lw;
   }
@@ -194,29 +196,39 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
     l_i[i] = r[0];
   }
 
-  // ---- o_d: thread (quarter qt, column d) folds slots [qt*SLOTS, +SLOTS)
-  // (a subtree) with the binary counter; the QT subtrees meet in order
-  const int d = tid % D, qt = tid / D;
-  float acc[G];
-  float lv[G][LV];
-#pragma unroll
-  for (int i = 0; i < G; i++) acc[i] = 0.0f;
+  // ---- o_d: thread (part qt, columns 2dp and 2dp + 1) folds slots
+  // [qt*SLOTS, +SLOTS) (a subtree) with the binary counter; one vector load
+  // gives every head's p of a slot; the QT subtrees meet in order
+  const int dp = tid % (D / 2), qt = tid / (D / 2);
+  float acc[G][2];
+  float lv[G][2][LV];
 #pragma unroll
   for (int s = 0; s < SLOTS; s++) {
     const int j = qt * SLOTS + s;
-    const float vv = j < nj ? __uint_as_float((uint32_t)s_v[j * D + d] << 16) : 0.0f;
+    const uint32_t vw = *reinterpret_cast<const uint32_t *>(&s_v[j * D + 2 * dp]);
+    const float v0 = j < nj ? bf16lo(vw) : 0.0f, v1 = j < nj ? bf16hi(vw) : 0.0f;
+    float pj[GP];
+#pragma unroll
+    for (int u = 0; u < GP; u += 4) {
+      const float4 q4 = *reinterpret_cast<const float4 *>(&s_pt[j][u]);
+      pj[u] = q4.x; pj[u + 1] = q4.y; pj[u + 2] = q4.z; pj[u + 3] = q4.w;
+    }
 #pragma unroll
     for (int i = 0; i < G; i++) {
-      const float prod = j < nj ? __fmul_rn(s_p[i][j], vv) : 0.0f;
-      acc[i] = counter_fold<LV>(s, prod, lv[i]);
+      acc[i][0] = counter_fold<LV>(s, j < nj ? __fmul_rn(pj[i], v0) : 0.0f, lv[i][0]);
+      acc[i][1] = counter_fold<LV>(s, j < nj ? __fmul_rn(pj[i], v1) : 0.0f, lv[i][1]);
     }
   }
 #pragma unroll
-  for (int i = 0; i < G; i++) s_half[i][qt][d] = acc[i];
+  for (int i = 0; i < G; i++) {
+    s_half[i][qt][2 * dp] = acc[i][0];
+    s_half[i][qt][2 * dp + 1] = acc[i][1];
+  }
   __syncthreads();
+  const int d = tid % D;
   float *wsb = p.ws + (((size_t)b * p.Hq + hk * G) * p.max_chunks + c) * (D + 2);
   const size_t head_stride = (size_t)p.max_chunks * (D + 2);
-  if (qt == 0) {
+  if (tid < D) {
 #pragma unroll
     for (int i = 0; i < G; i++) {
       float r[QT];
