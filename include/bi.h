@@ -300,6 +300,18 @@ bi_status bi_get_device_status(bi_stream_t stream);
 /* Human-readable name of a status code (static string). */
 const char *bi_status_string(int status);
 
+/* Test-only fault injection on the host side.  With fault_code =
+ * BI_FAULT_SKIP_STAGE every following bi_gemm / bi_addmm call runs with the
+ * TMA producer of its first CTA leaving the first K stage unloaded: the MMA
+ * issuer's bounded wait on that stage runs out, the kernel records
+ * BI_ERR_TIMEOUT, waits (bounded) for every load and MMA it did issue, frees
+ * its tensor memory and returns, so the context stays usable.  While a
+ * fault is set the kernels' waits give up after 10 ms instead of 2 s.
+ * fault_code = 0 (BI_FAULT_NONE) turns it off.  No GPU fault is involved. */
+#define BI_FAULT_NONE 0
+#define BI_FAULT_SKIP_STAGE 1
+void bi_debug_set_fault(int fault_code);
+
 /* Self-test of the bounded-wait machinery: launches one CTA that waits on
  * a flag nothing sets, giving up after `max_polls` polls; the kernel then
  * records BI_ERR_TIMEOUT in the device status word and returns.  Used to

@@ -57,6 +57,7 @@ _SIGS = {
     "bi_get_device_status": (I, [P]),
     "bi_status_string": (ctypes.c_char_p, [I]),
     "bi_selftest_bounded_wait": (I, [I, P]),
+    "bi_debug_set_fault": (None, [I]),
 }
 
 
@@ -394,3 +395,13 @@ def status_string(code: int) -> str:
 
 def selftest_bounded_wait(max_polls=1000, stream=None):
     _call("bi_selftest_bounded_wait", int(max_polls), _stream(stream))
+
+
+FAULT_NONE, FAULT_SKIP_STAGE = 0, 1
+
+
+def debug_set_fault(code):
+    """Test-only: FAULT_SKIP_STAGE makes the following GEMM calls leave one
+    stage unloaded (their bounded wait reports BI_ERR_TIMEOUT); FAULT_NONE
+    turns it off."""
+    lib().bi_debug_set_fault(int(code))

@@ -31,6 +31,7 @@
 #include "tc.cuh"
 
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <mutex>
 
 namespace bi {
@@ -56,15 +57,24 @@ struct GemmSmemTail {
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t drain;            // the MMA issuer's last commit, before TMEM is freed
   uint32_t tmem_base;
   uint32_t bail;
+};
+
+// Test-only fault (bi_debug_set_fault): the producer of CTA 0 leaves the
+// first stage of its first tile unloaded, so the MMA issuer's wait on it
+// runs out; waits then give up after wait_ns.
+struct GemmDebug {
+  int fault;
+  unsigned long long wait_ns;
 };
 
 template <int BN>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  void *__restrict__ C, const uint16_t *__restrict__ bias, int M, int N, int K, int c_bf16,
-                 unsigned *status) {
+                 unsigned *status, GemmDebug dbg) {
   using namespace gemm;
   constexpr int STAGES = Cfg<BN>::STAGES, B_BYTES = Cfg<BN>::B_BYTES, STAGE_BYTES = Cfg<BN>::STAGE_BYTES;
   constexpr uint32_t TMEM_COLS = Cfg<BN>::TMEM_COLS;
@@ -88,6 +98,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&tail->tfull[b], 1);
       mbar_init(&tail->tempty[b], 4);
     }
+    mbar_init(&tail->drain, 1);
     tail->bail = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
@@ -107,20 +118,33 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       // ---------------- TMA producer
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;             // per stage: loads in flight, and their phase
       for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
         const int mb = tile % tiles_m, nb = tile / tiles_m;
         for (int kb = 0; kb < kblocks; kb++) {
-          if (!mbar_wait(&tail->empty[stage], phase ^ 1)) {
+          if (!mbar_wait_for(&tail->empty[stage], phase ^ 1, dbg.wait_ns)) {
             flag_error(status, BI_ERR_TIMEOUT);
             *bail = 1;
             break;
           }
-          mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
-          tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, kb * BK, mb * BM);
-          tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, kb * BK, nb * BN);
+          const bool skip = dbg.fault == BI_FAULT_SKIP_STAGE && blockIdx.x == 0 && tile == (int)blockIdx.x && kb == 0;
+          if (!skip) {
+            mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
+            tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, kb * BK, mb * BM);
+            tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, kb * BK, nb * BN);
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          } else {
+            issued &= ~(1u << stage);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // every load issued has landed before the CTA's shared memory is
+      // given up (a stage the MMAs consumed passes at once)
+      for (int s = 0; s < STAGES; s++)
+        if ((issued >> s) & 1u)
+          if (!mbar_wait_for(&tail->full[s], (issued_par >> s) & 1u, dbg.wait_ns)) flag_error(status, BI_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -131,7 +155,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
-        if (!mbar_wait(&tail->tempty[acc], acc_phase ^ 1)) {
+        if (!mbar_wait_for(&tail->tempty[acc], acc_phase ^ 1, dbg.wait_ns)) {
           flag_error(status, BI_ERR_TIMEOUT);
           *bail = 1;
           break;
@@ -139,7 +163,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < kblocks; kb++) {
-          if (!mbar_wait(&tail->full[stage], phase)) {
+          if (!mbar_wait_for(&tail->full[stage], phase, dbg.wait_ns)) {
             flag_error(status, BI_ERR_TIMEOUT);
             *bail = 1;
             break;
@@ -157,6 +181,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         umma_commit(&tail->tfull[acc]);              // accumulator ready for the epilogue
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
+      // every MMA issued has completed before TMEM is freed
+      umma_commit(&tail->drain);
+      if (!mbar_wait_for(&tail->drain, 0, dbg.wait_ns)) flag_error(status, BI_ERR_TIMEOUT);
     }
   } else {
     // ---------------- epilogue: 4 warps, one TMEM lane quadrant each
@@ -166,7 +193,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       if (*bail) break;
-      if (!mbar_wait(&tail->tfull[acc], acc_phase)) {
+      if (!mbar_wait_for(&tail->tfull[acc], acc_phase, dbg.wait_ns)) {
         flag_error(status, BI_ERR_TIMEOUT);
         *bail = 1;
         break;
@@ -270,6 +297,8 @@ int num_sms() {
   return cache[dev];
 }
 
+static std::atomic<int> g_fault{0};
+
 template <int BN>
 static bi_status gemm_run(const void *A, const void *W, void *C, const void *bias, int M, int N, int K, int c_bf16,
                           cudaStream_t stream) {
@@ -285,8 +314,9 @@ static bi_status gemm_run(const void *A, const void *W, void *C, const void *bia
     return BI_ERR_CUDA;
   const long tiles = (long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<long>(tiles, num_sms());
+  GemmDebug dbg{g_fault.load(), g_fault.load() ? 10000000ull : kWaitLimitNs};
   gemm_bf16_kernel<BN><<<grid, THREADS, SMEM, stream>>>(tmA, tmW, C, static_cast<const uint16_t *>(bias), M, N, K,
-                                                       c_bf16 ? 1 : 0, status_word());
+                                                       c_bf16 ? 1 : 0, status_word(), dbg);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
@@ -317,3 +347,5 @@ extern "C" bi_status bi_addmm(const void *bias, const void *A, const void *W, vo
   if (M > 0 && !bias) return BI_ERR_INVALID_ARG;
   return bi::gemm_launch(A, W, C, bias, M, N, K, c_bf16, reinterpret_cast<cudaStream_t>(stream));
 }
+
+extern "C" void bi_debug_set_fault(int fault_code) { bi::g_fault.store(fault_code); }

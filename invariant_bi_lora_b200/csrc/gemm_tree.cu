@@ -66,6 +66,7 @@ struct TreeSmemTail {
   uint64_t empty[tg::MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t drain;            // the MMA issuer's last commit, before TMEM is freed
   uint32_t tmem_base;
   uint32_t bail;
 };
@@ -112,6 +113,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(&tail->tfull[b], 1);
       mbar_init(&tail->tempty[b], EPI_WARPS);
     }
+    mbar_init(&tail->drain, 1);
     tail->bail = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
@@ -138,6 +140,7 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;           // per stage: loads in flight, and their phase
       for (int tile = blockIdx.x; tile < num_tiles && !*bail; tile += gridDim.x) {
         int mb, nb, sh;
         decode(tile, mb, nb, sh);
@@ -151,9 +154,16 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
           tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, (kb0 + kb) * BK, mb * BM);
           tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, (kb0 + kb) * BK, nb * BN);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // every load issued has landed before the CTA's shared memory is
+      // given up (a stage the MMAs consumed passes at once)
+      for (int s = 0; s < STAGES; s++)
+        if ((issued >> s) & 1u)
+          if (!mbar_wait(&tail->full[s], (issued_par >> s) & 1u)) flag_error(p.status, BI_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -191,6 +201,9 @@ gemm_tree_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (++buf == NBUF) { buf = 0; buf_phase ^= 1; }
         }
       }
+      // every MMA issued has completed before TMEM is freed
+      umma_commit(&tail->drain);
+      if (!mbar_wait(&tail->drain, 0)) flag_error(p.status, BI_ERR_TIMEOUT);
     }
   } else if constexpr (LPS == 0) {
     // ---------------- epilogue: post-order fold of the leaves, stack in TMEM

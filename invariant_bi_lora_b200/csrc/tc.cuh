@@ -58,16 +58,17 @@ BI_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase of the given parity; false if the bound ran out.
-BI_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
+BI_DEV bool mbar_wait_for(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 64; i++)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
+BI_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitLimitNs); }
 
 // ------------------------------------------------------------------ TMA
 // 2-D tile load into shared memory, completion counted on `bar` (bytes).
