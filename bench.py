@@ -777,10 +777,10 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------- one-op cases (ncu)
 
-CASES = ("plan", "shrink", "shrink_segmented", "expand_segmented", "gemm", "tree_gemm", "rmsnorm",
-         "log_softmax", "mean")
+CASES = ("plan", "shrink", "shrink_segmented", "expand_segmented", "fused", "gemm", "addmm", "tree_gemm",
+         "attn_decode", "rmsnorm", "log_softmax", "mean")
 CASE_DEFAULTS = {"M": 16384, "K": 4096, "N": 4096, "r": 16, "adapters": 8, "splits": 8, "mode": "tree",
-                 "shards": 8, "rows": 4096, "n": 151936}
+                 "shards": 8, "rows": 4096, "n": 151936, "B": 32, "L": 2048, "Hq": 32, "Hkv": 8, "D": 128}
 
 
 def run_case(a):
@@ -790,9 +790,9 @@ def run_case(a):
     from invariant_bi_lora_b200 import bi, synth
     torch.cuda.set_device(0)
     op = a.case
-    if op in ("plan", "shrink", "shrink_segmented", "expand_segmented"):
+    if op in ("plan", "shrink", "shrink_segmented", "expand_segmented", "fused"):
         d = synth.lora_inputs(a.M, a.K, a.r, n_adapters=a.adapters,
-                              N=a.N if op == "expand_segmented" else 0, seed=0)
+                              N=a.N if op in ("expand_segmented", "fused") else 0, seed=0)
         X, A = dev_bf16(d["x"]), dev_bf16(d["at"])
         y = torch.empty(a.M, a.r, dtype=torch.float32, device="cuda")
         ids = torch.from_numpy(d["ids"]).cuda()
@@ -804,20 +804,36 @@ def run_case(a):
             run = lambda: bi.lora_shrink(X, A0, y, a.splits, a.mode)
         elif op == "shrink_segmented":
             run = lambda: bi.lora_shrink_segmented(X, A, plan, y, a.splits, a.mode)
+        elif op == "fused":
+            B = dev_bf16(d["bt"])
+            out = torch.empty(a.M, a.N, dtype=torch.float32, device="cuda")
+            run = lambda: bi.lora_fused(X, A, B, plan, out, splits=a.splits)
         else:
             B = dev_bf16(d["bt"])
             out = torch.empty(a.M, a.N, dtype=torch.float32, device="cuda")
             bi.lora_shrink_segmented(X, A, plan, y, a.splits, "tree")
             run = lambda: bi.lora_expand_segmented(y, B, plan, out)
-    elif op in ("gemm", "tree_gemm"):
+    elif op in ("gemm", "addmm", "tree_gemm"):
         g_a, g_w = synth.gemm_inputs(a.M, a.N, a.K, seed=0)
         GA, GW = dev_bf16(g_a), dev_bf16(g_w)
         C = torch.empty(a.M, a.N, dtype=torch.float32, device="cuda")
         if op == "gemm":
             run = lambda: bi.gemm(GA, GW, C)
+        elif op == "addmm":
+            bias = dev_bf16(synth.normal_bf16((a.N,), 1.0, seed=0, tag=9))
+            run = lambda: bi.addmm(bias, GA, GW, C)
         else:
             ws = torch.empty(max(1, bi.gemm_tree_ws_bytes(a.M, a.N, a.shards)), dtype=torch.uint8, device="cuda")
             run = lambda: bi.gemm_tree(GA, GW, C, a.shards, ws)
+    elif op == "attn_decode":
+        gen = torch.Generator().manual_seed(0)
+        q = torch.randn(a.B, a.Hq, a.D, generator=gen).to(torch.bfloat16).cuda()
+        kk = torch.randn(a.B, a.Hkv, a.L, a.D, generator=gen).to(torch.bfloat16).cuda()
+        vv = torch.randn(a.B, a.Hkv, a.L, a.D, generator=gen).to(torch.bfloat16).cuda()
+        lens = torch.full((a.B,), a.L, dtype=torch.int32, device="cuda")
+        out = torch.empty(a.B, a.Hq, a.D, dtype=torch.float32, device="cuda")
+        ws = torch.empty(bi.attn_decode_ws_bytes(a.B, a.Hq, a.D, a.L), dtype=torch.uint8, device="cuda")
+        run = lambda: bi.attn_decode(q, kk, vv, lens, out, ws=ws)
     elif op == "rmsnorm":
         x, w = synth.rmsnorm_inputs(a.rows, a.n, seed=0)
         X, W = dev_bf16(x), dev_bf16(w)
