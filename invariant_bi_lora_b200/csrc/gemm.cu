@@ -43,11 +43,24 @@ constexpr int A_BYTES = BM * BK * 2;                  // 16 KB
 // Per output-tile width BN: the W stage, the ring depth, TMEM columns.
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = BN >= 256 ? 4 : 8;
+  static constexpr int STAGES = BN >= 256 ? 4 : 8;   // with full 128-row A stages
+  static constexpr int MAX_STAGES = BN == 32 ? 32 : STAGES;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;   // two accumulators
-  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+};
+// The ring of one launch.  At M <= 64 the A box holds only a_rows =
+// round_up(M, 8) rows, so a stage is mostly W and the ring can be deep; the
+// MMA still reads a 128-row A window from each stage's start, whose rows
+// past a_rows fall on the next stages (or on the slack after the ring) and
+// produce output rows that are never stored: a row of an MMA's result
+// depends on that row of A only.
+struct GemmRing {
+  int stages;        // ring depth
+  int a_rows;        // rows of the A box (128, or round_up(M, 8) at M <= 64)
+  int a_stage;       // bytes between A stages (a_rows * 128)
+  int b_off;         // bytes from the ring start to the W stages
+  int tail_off;      // bytes from the ring start to the barriers
 };
 }  // namespace gemm
 
@@ -74,15 +87,18 @@ template <int BN>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  void *__restrict__ C, const uint16_t *__restrict__ bias, int M, int N, int K, int c_bf16,
-                 unsigned *status, GemmDebug dbg) {
+                 unsigned *status, GemmDebug dbg, gemm::GemmRing ring) {
   using namespace gemm;
-  constexpr int STAGES = Cfg<BN>::STAGES, B_BYTES = Cfg<BN>::B_BYTES, STAGE_BYTES = Cfg<BN>::STAGE_BYTES;
+  constexpr int MAXST = Cfg<BN>::MAX_STAGES, B_BYTES = Cfg<BN>::B_BYTES;
   constexpr uint32_t TMEM_COLS = Cfg<BN>::TMEM_COLS;
+  const int STAGES = ring.stages;
+  const int A_STAGE = ring.a_stage;
+  const uint32_t STAGE_TX = (uint32_t)(ring.a_rows * BK * 2 + B_BYTES);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sa = smem;                                 // [STAGES][A_BYTES]
-  uint8_t *sb = smem + STAGES * A_BYTES;              // [STAGES][B_BYTES]
-  GemmSmemTail<STAGES> *tail = reinterpret_cast<GemmSmemTail<STAGES> *>(smem + STAGES * STAGE_BYTES);
+  uint8_t *sa = smem;                                 // [STAGES][A_STAGE] + slack
+  uint8_t *sb = smem + ring.b_off;                    // [STAGES][B_BYTES]
+  GemmSmemTail<MAXST> *tail = reinterpret_cast<GemmSmemTail<MAXST> *>(smem + ring.tail_off);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
@@ -129,8 +145,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
           const bool skip = dbg.fault == BI_FAULT_SKIP_STAGE && blockIdx.x == 0 && tile == (int)blockIdx.x && kb == 0;
           if (!skip) {
-            mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
-            tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_BYTES, kb * BK, mb * BM);
+            mbar_arrive_expect_tx(&tail->full[stage], STAGE_TX);
+            tma_load_2d(&tmA, &tail->full[stage], sa + stage * A_STAGE, kb * BK, mb * BM);
             tma_load_2d(&tmW, &tail->full[stage], sb + stage * B_BYTES, kb * BK, nb * BN);
             issued |= 1u << stage;
             issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -169,7 +185,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sa + stage * A_BYTES);
+          const uint32_t a0 = smem_u32(sa + stage * A_STAGE);
           const uint32_t b0 = smem_u32(sb + stage * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; k++)
@@ -303,10 +319,22 @@ template <int BN>
 static bi_status gemm_run(const void *A, const void *W, void *C, const void *bias, int M, int N, int K, int c_bf16,
                           cudaStream_t stream) {
   using namespace gemm;
+  GemmRing ring{};
+  ring.a_rows = (BN == 32 && M <= 64) ? ((M + 7) & ~7) : BM;
+  ring.a_stage = ring.a_rows * BK * 2;
+  const int slack = (BM - ring.a_rows) * BK * 2;     // the last stage's 128-row window
+  if (ring.a_rows < BM) {
+    const int budget = 200 * 1024 - slack;
+    ring.stages = std::min(Cfg<BN>::MAX_STAGES, budget / (ring.a_stage + Cfg<BN>::B_BYTES));
+  } else {
+    ring.stages = Cfg<BN>::STAGES;
+  }
+  ring.b_off = (ring.stages * ring.a_stage + slack + 1023) & ~1023;
+  ring.tail_off = ring.b_off + ring.stages * Cfg<BN>::B_BYTES;
+  const size_t SMEM = 1024 + (size_t)ring.tail_off + sizeof(GemmSmemTail<Cfg<BN>::MAX_STAGES>);
   CUtensorMap tmA, tmW;
-  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, BM)) return BI_ERR_CUDA;
+  if (!make_tma_2d_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, BK, (uint32_t)ring.a_rows)) return BI_ERR_CUDA;
   if (!make_tma_2d_bf16(&tmW, W, (uint64_t)K, (uint64_t)N, BK, BN)) return BI_ERR_CUDA;
-  constexpr size_t SMEM = Cfg<BN>::SMEM;
   // per launch: the attribute belongs to the current device, and a process
   // may drive several
   if (cudaFuncSetAttribute(gemm_bf16_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM) !=
@@ -316,7 +344,7 @@ static bi_status gemm_run(const void *A, const void *W, void *C, const void *bia
   const int grid = (int)std::min<long>(tiles, num_sms());
   GemmDebug dbg{g_fault.load(), g_fault.load() ? 10000000ull : kWaitLimitNs};
   gemm_bf16_kernel<BN><<<grid, THREADS, SMEM, stream>>>(tmA, tmW, C, static_cast<const uint16_t *>(bias), M, N, K,
-                                                       c_bf16 ? 1 : 0, status_word(), dbg);
+                                                       c_bf16 ? 1 : 0, status_word(), dbg, ring);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -174,8 +174,10 @@ mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
 // [q*4096/C, (q+1)*4096/C) -- a subtree of the lane tree -- one thread per
 // lane, each keeping its lane's vectors in shared memory (slot [j][tau] for
 // vector 4096*j + lane).  Maxima and sums meet through distributed shared
-// memory.  The sum pass stores d = x - max back into the slot, so the write
-// pass is one subtraction per element.
+// memory: each CTA pushes its value into a slot of every CTA of the cluster
+// before a barrier, so after it every CTA reads only its own shared memory
+// and no CTA waits for its peers at exit.  The sum pass stores d = x - max
+// back into the slot, so the write pass is one subtraction per element.
 // ======================================================================
 constexpr int kLsmT = 4096;
 
@@ -221,7 +223,8 @@ __global__ void __launch_bounds__(THREADS, THREADS == 256 ? 5 : 0)
 log_softmax_kernel(const __grid_constant__ LsmParams p) {
   extern __shared__ float4 lsm_smem[];
   __shared__ float s_red[32];
-  __shared__ float s_max, s_sum, s_bcast, s_bcast2;
+  __shared__ float s_max, s_sum;
+  __shared__ float s_maxs[16], s_sums[16];     // the cluster's values, pushed by their owners
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C;
   const int q = (int)cluster.block_rank();
@@ -235,6 +238,10 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   const int nwarps = lpc / 32;
   // this lane's vectors: 4096*j + lane_id for j < nj
   const int nj = lane_id < nvec ? (nvec - 1 - lane_id) / kLsmT + 1 : 0;
+
+  // every CTA of the cluster has started once this arrive is matched; the
+  // wait comes before the first write into a peer's shared memory
+  cluster_arrive_relaxed();
 
   // ---- this lane's vectors -> its shared-memory slots: 16-byte cp.async
   // copies, all in flight at once.  Each thread reads back only its own
@@ -256,16 +263,16 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     v = warp_max(v);
     if (tau == 0) s_max = v;
   }
+  __syncthreads();
+  cluster_wait();
+  // push this CTA's max into slot q of every CTA of the cluster
+  if (tau < C) *cluster.map_shared_rank(&s_maxs[q], tau) = s_max;
   cluster_arrive_release();
   cluster_wait_acquire();
-  // row max over the cluster (exact in any order): warp 0 gathers, all read
-  if (tau < 32) {
-    float v = tau < C ? *cluster.map_shared_rank(&s_max, tau) : -INFINITY;
-    v = warp_max(v);
-    if (tau == 0) s_bcast = v;
-  }
-  __syncthreads();
-  const uint64_t rmax2 = splat2(s_bcast);
+  // row max over the cluster (exact in any order), from this CTA's own slots
+  float rmax = s_maxs[0];
+  for (int t = 1; t < C; t++) rmax = fmaxf(rmax, s_maxs[t]);
+  const uint64_t rmax2 = splat2(rmax);
 
   // ---- lane chain of bi_exp(x - max); d = x - max stays in the slot
   float s = 0.0f;
@@ -290,18 +297,19 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     for (int o = 1; o < nwarps; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
     if (tau == 0) s_sum = v;
   }
+  __syncthreads();
+  // push this CTA's subtree value into slot q of every CTA; after the
+  // barrier nothing reads or writes a peer's memory, so no CTA waits for the
+  // others before it exits
+  if (tau < C) *cluster.map_shared_rank(&s_sums[q], tau) = s_sum;
   cluster_arrive_release();
   cluster_wait_acquire();
-  // perfect tree over the C CTA subtrees: warp 0 gathers them into lanes
-  // 0..C-1 and adds with the xor butterfly (pairs, then pairs of pairs)
-  if (tau < 32) {
-    float v = tau < C ? *cluster.map_shared_rank(&s_sum, tau) : 0.0f;
-    for (int o = 1; o < C; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (tau == 0) s_bcast2 = bi_log(v);
-  }
-  __syncthreads();
-  cluster_arrive_relaxed();               // done reading the peers' shared memory
-  const uint64_t L2 = splat2(s_bcast2);
+  // perfect tree over the C CTA subtrees (lanes 0..C-1, xor butterfly:
+  // pairs, then pairs of pairs); every warp computes it from its own copy
+  float v = (tau & 31) < C ? s_sums[tau & 31] : 0.0f;
+  for (int o = 1; o < C; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  v = __shfl_sync(0xffffffffu, v, 0);           // lanes >= C added zeros among themselves
+  const uint64_t L2 = splat2(bi_log(v));
 
   // ---- write out = d - L
   for (int j = 0; j < nj; j++) {
@@ -311,7 +319,6 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     const float4 o = make_float4(o01.x, o01.y, o23.x, o23.y);
     __stcs(outr + (size_t)j * kLsmT + lane_id, o);
   }
-  cluster_wait();                         // keep s_max / s_sum alive until the peers are done
 }
 
 // Test and reference hook: the library's exp / log applied elementwise.
