@@ -212,8 +212,13 @@ bi_status bi_addmm(const void *bias, const void *A, const void *W, void *C, int 
 /* levels.  The result is bitwise the same for shards = 1, 2, 4, 8, 16. */
 /*                                                                      */
 /* bi_gemm_tree_partials: partials fp32 [shards][M][N].                */
-/* bi_gemm_tree: C fp32 [M][N]; for shards > 1 it needs a workspace of  */
-/*   bi_gemm_tree_ws_bytes(M, N, shards) bytes (the partials).          */
+/* bi_gemm_tree: C fp32 [M][N]; workspace of                            */
+/*   bi_gemm_tree_ws_bytes(M, N, shards) bytes for the partials (at     */
+/*   least four, so that a shard of 32 or 64 leaves can be folded as    */
+/*   power-of-two subtrees of 16 leaves and combined: same bits, faster */
+/*   layout).  shards = 1 also runs without a workspace (ws = NULL),    */
+/*   folding all leaves in one partial; shards > 1 needs at least       */
+/*   shards * M * N * 4 bytes.                                          */
 /* Requirements: K % 256 == 0, shards a power of two dividing K/256,    */
 /* N % 64 == 0, pointers 16-byte aligned.                               */
 /* ------------------------------------------------------------------ */

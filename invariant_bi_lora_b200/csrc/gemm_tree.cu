@@ -419,9 +419,17 @@ static bi_status tree_partials_launch(const void *A, const void *W, float *out, 
 
 }  // namespace bi
 
+// Workspace of bi_gemm_tree: the partials of the schedule it runs.  Every
+// power-of-two cut of the leaves that divides their count is a cut into
+// subtrees of the canonical tree, so the final C is the same bits whether
+// the tree over a shard's leaves is folded in one partial or in several that
+// a combine then adds; with up to 16 leaves per partial the kernel folds on
+// its fast layout.  The size returned covers four partials at least, enough
+// for K <= 16384 (64 leaves) at any shard count; with less, the call folds
+// each shard's leaves in one partial (slower for 32 or 64 leaves a shard).
 extern "C" size_t bi_gemm_tree_ws_bytes(int M, int N, int shards) {
-  if (M < 0 || N < 0 || shards <= 1) return 0;
-  return sizeof(float) * (size_t)shards * M * N;
+  if (M < 0 || N < 0 || shards < 1) return 0;
+  return sizeof(float) * (size_t)std::max(shards, 4) * M * N;
 }
 
 extern "C" bi_status bi_gemm_tree_partials(const void *A, const void *W, float *partials, int M, int N, int K,
@@ -441,12 +449,19 @@ extern "C" bi_status bi_gemm_tree(const void *A, const void *W, float *C, int M,
   if (M > 0 && !bi_aligned16(C)) return BI_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return BI_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (shards == 1) return bi::tree_partials_launch(A, W, C, M, N, K, 1, s);
-  const size_t need = bi_gemm_tree_ws_bytes(M, N, shards);
+  // partials: the shards, cut further (power-of-two subtrees) until each
+  // holds at most 16 leaves, when the workspace allows it
+  const int L = K / bi::tg::LEAF;
+  int P = shards;
+  while (L / P > 16 && L % (2 * P) == 0 && 2 * P <= bi::tg::MAX_LEAVES) P *= 2;
+  const size_t fast = sizeof(float) * (size_t)P * M * N;
+  if (P > shards && (!ws || ws_bytes < fast || !bi_aligned16(ws))) P = shards;
+  if (P == 1) return bi::tree_partials_launch(A, W, C, M, N, K, 1, s);
+  const size_t need = sizeof(float) * (size_t)P * M * N;
   if (!ws || ws_bytes < need) return BI_ERR_WORKSPACE;
   if (!bi_aligned16(ws)) return BI_ERR_UNSUPPORTED_SHAPE;
   float *parts = static_cast<float *>(ws);
-  st = bi::tree_partials_launch(A, W, parts, M, N, K, shards, s);
+  st = bi::tree_partials_launch(A, W, parts, M, N, K, P, s);
   if (st != BI_OK) return st;
-  return bi::tree_combine_launch(parts, C, shards, (size_t)M * N, s);
+  return bi::tree_combine_launch(parts, C, P, (size_t)M * N, s);
 }
