@@ -21,6 +21,10 @@
 // same warp aggregation), so the segment offsets are known before the
 // scatter.
 #include "common.cuh"
+#include "tc.cuh"
+
+#include <algorithm>
+#include <cooperative_groups.h>
 
 namespace bi {
 
@@ -65,96 +69,135 @@ BI_DEV void plan_rank(const int (&cls)[kPlanPer], int *mine, int ncls, int lane,
   }
 }
 
-// At most 32 classes and at most one chunk (n_ad <= 31, M <= 4096), the
-// common serving case: a single pass with two block barriers.  A warp
-// ranks its tokens with one ballot per class and j (no shared-memory
-// atomics, no match), lane c of the warp records the warp's count of class
-// c, and warp 0 alone turns the 32 x ncls counts into warp bases, segment
-// starts and table bases (ncls lanes, a shuffle scan).
-__global__ void __launch_bounds__(kPlanThreads, 1)
+// At most 32 classes and at most 4096 tokens (n_ad <= 31), the common
+// serving case: one cluster of ceil(M / 512) CTAs of 4 warps, a warp per
+// 128 tokens, so that the rank work of up to 32 warps runs on up to 8 SMs.
+//  * Rank: a class fits in nb <= 5 bits, so one ballot per bit of the
+//    j-th tokens gives every lane both the lanes whose token shares its
+//    class (the AND of the bit masks, complemented where its bit is 0) and,
+//    for lane c, the lanes whose token has class c.  Lane c keeps the
+//    warp's running count of class c; a token's rank is that count (read
+//    from lane cls by shuffle) plus its same-class lanes below it.
+//  * Bases: every warp pushes its row of class counts into every CTA's
+//    [warp][class] table (distributed shared memory), and after one
+//    cluster barrier each warp scans the whole table itself (lane c: its
+//    class's count in the warps before this one and in all warps; a
+//    shuffle scan over the lanes gives the segment starts and table bases).
+//  * Table: records are written as 17 16-byte quads (header, 16 quads of
+//    token slots), spread over all threads; a slot quad is written only
+//    where it holds unused (-1) slots, the scatter fills the rest.
+constexpr int kPlanSmallWarps = 4;                  // per CTA
+constexpr int kPlanSmallCtas = 8;                   // per cluster: 8 * 4 * 128 = 4096 tokens
+constexpr int kPlanQuads = kPlanRec / 4;            // 17
+
+__global__ void __launch_bounds__(32 * kPlanSmallWarps)
 plan_small_kernel(const int32_t *__restrict__ ids, int M, int n_ad, int32_t *__restrict__ plan) {
-  __shared__ int wc[kPlanWarps][33];     // warp counts, then warp bases
-  __shared__ int s_off[33], s_tbase[33], s_cnt[33];
-  const int ncls = n_ad + 1;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ int wc[kPlanSmallCtas * kPlanSmallWarps][32];   // warp w's count of class c
+  const int ncls = n_ad + 1, ncta = gridDim.x;       // the grid is one cluster
+  const int lane = threadIdx.x & 31;
+  const int warp = blockIdx.x * kPlanSmallWarps + (threadIdx.x >> 5), nw = ncta * kPlanSmallWarps;
   const unsigned lt_mask = (1u << lane) - 1u;
   int32_t *perm = plan;
   int32_t *offsets = plan + M;
   int32_t *table = plan + plan_table_word(M, n_ad);
   const int ntiles = (int)plan_tiles(M, n_ad);
+  // every CTA has started once this arrive is matched; the wait comes
+  // before the first write into a peer's shared memory
+  cluster_arrive_relaxed();
+  // start the output's address translation while the ids are in flight
+  if (warp == 0 && lane == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(plan));
+  if (warp == nw - 1 && lane == 0)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(table + (size_t)ntiles * kPlanRec - 1));
 
   int cls[kPlanPer];
   plan_load(ids, M, n_ad, 0, warp, lane, cls);
-  int rank[kPlanPer] = {0, 0, 0, 0};
-  int mycount = 0;                                    // lane c: the warp's tokens of class c
-  for (int c = 0; c < ncls; c++) {
-    int run = 0;
+  const int nb = 32 - __clz(ncls - 1);                // bits of the largest class, 1..5
+  int rank[kPlanPer];
+  int run = 0;                                        // lane c: the warp's tokens of class c so far
 #pragma unroll
-    for (int j = 0; j < kPlanPer; j++) {
-      const unsigned m = __ballot_sync(0xffffffffu, cls[j] == c);
-      if (cls[j] == c) rank[j] = run + __popc(m & lt_mask);
-      run += __popc(m);
-    }
-    if (lane == c) mycount = run;
-  }
-  if (lane < ncls) wc[warp][lane] = mycount;
-  __syncthreads();
-  if (warp == 0) {
-    // lane c: its class's warp bases (in place) and total
-    int total = 0;
-    if (lane < ncls) {
-#pragma unroll 8
-      for (int w = 0; w < kPlanWarps; w++) {
-        const int n = wc[w][lane];
-        wc[w][lane] = total;
-        total += n;
+  for (int j = 0; j < kPlanPer; j++) {
+    unsigned same = __ballot_sync(0xffffffffu, cls[j] >= 0), mine = same;
+#pragma unroll
+    for (int bit = 0; bit < 5; bit++) {
+      if (bit < nb) {
+        const unsigned m = __ballot_sync(0xffffffffu, (cls[j] >> bit) & 1);
+        same &= ((cls[j] >> bit) & 1) ? m : ~m;
+        mine &= ((lane >> bit) & 1) ? m : ~m;
       }
     }
-    const int tv = (total + kPlanTile - 1) / kPlanTile;
-    int vin = total, tin = tv;
+    rank[j] = __shfl_sync(0xffffffffu, run, cls[j] & 31) + __popc(same & lt_mask);
+    run += __popc(mine);
+  }
+  const int mycount = lane < ncls ? run : 0;
+  cluster_wait();
+  for (int r = 0; r < ncta; r++) *cluster.map_shared_rank(&wc[warp][lane], r) = mycount;
+  cluster_arrive_release();
+  cluster_wait_acquire();
+
+  int before = 0, total = 0;                          // lane c: class c in warps < this one, in all
+#pragma unroll 8
+  for (int w = 0; w < nw; w++) {
+    const int n = wc[w][lane];
+    before += w < warp ? n : 0;
+    total += n;
+  }
+  const int tv = (total + kPlanTile - 1) / kPlanTile;
+  int vin = total, tin = tv;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, vin, o), b = __shfl_up_sync(0xffffffffu, tin, o);
-      if (lane >= o) vin += a, tin += b;
-    }
-    if (lane < ncls) {
-      s_off[lane] = vin - total;
-      s_tbase[lane] = tin - tv;
-      s_cnt[lane] = total;
-      offsets[lane] = vin - total;
-    }
-    if (lane == ncls - 1) {
-      s_off[ncls] = vin;
-      s_tbase[ncls] = tin;
-      offsets[ncls] = vin;
-    }
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, vin, o), y = __shfl_up_sync(0xffffffffu, tin, o);
+    if (lane >= o) vin += x, tin += y;
+  }
+  // lane c: segment start and first record of class c (lanes >= ncls: the
+  // totals, so the table bases stay non-decreasing over all 32 lanes)
+  const int off = vin - total, tbase = tin - tv;
+  const int used = __shfl_sync(0xffffffffu, tin, 31);
+  if (warp == 0) {
+    if (lane < ncls) offsets[lane] = off;
+    if (lane == ncls - 1) offsets[ncls] = vin;
     if (lane < plan_table_word(M, n_ad) - (M + ncls + 1)) plan[M + ncls + 1 + lane] = 0;   // padding
   }
-  __syncthreads();
-  // table headers and the unused id slots, one warp per record
-  const int used = s_tbase[ncls];
-  for (int i = warp; i < ntiles; i += kPlanWarps) {
-    int a = -1, rows = 0, first = 0;
-    if (i < used) {
-      int lo = 0;
-      while (lo + 1 < ncls && s_tbase[lo + 1] <= i) lo++;
-      const int j = i - s_tbase[lo];
-      a = lo;
-      rows = min(kPlanTile, s_cnt[lo] - kPlanTile * j);
-      first = s_off[lo] + kPlanTile * j;
-    }
-    int32_t *rec = table + (size_t)i * kPlanRec;
-    if (lane == 0) *reinterpret_cast<int4 *>(rec) = make_int4(a, rows, first, 0);
-    for (int s = rows + lane; s < kPlanTile; s += 32) rec[4 + s] = -1;
-  }
+
   // stable scatter
 #pragma unroll
   for (int j = 0; j < kPlanPer; j++) {
+    const int c = cls[j] & 31;
+    const int sp = __shfl_sync(0xffffffffu, before, c) + rank[j];   // position inside the segment
+    const int o = __shfl_sync(0xffffffffu, off, c), tb = __shfl_sync(0xffffffffu, tbase, c);
     if (cls[j] < 0) continue;
     const int t = warp * (32 * kPlanPer) + 32 * j + lane;
-    const int sp = wc[warp][cls[j]] + rank[j];          // position inside the segment
-    perm[s_off[cls[j]] + sp] = t;
-    table[(size_t)(s_tbase[cls[j]] + sp / kPlanTile) * kPlanRec + 4 + sp % kPlanTile] = t;
+    perm[o + sp] = t;
+    table[(size_t)(tb + sp / kPlanTile) * kPlanRec + 4 + sp % kPlanTile] = t;
+  }
+  // table records: quad q of record i is item 17 i + q
+  const int items = ntiles * kPlanQuads;
+  for (int base = 32 * warp; base < items; base += 32 * nw) {
+    const int it = base + lane, i = it / kPlanQuads, q = it - kPlanQuads * i;
+    int c = 0;                                        // largest class whose first record is <= i
+#pragma unroll
+    for (int step = 16; step; step >>= 1)
+      if (__shfl_sync(0xffffffffu, tbase, c + step) <= i) c += step;
+    const int tb = __shfl_sync(0xffffffffu, tbase, c), o = __shfl_sync(0xffffffffu, off, c);
+    const int cnt = __shfl_sync(0xffffffffu, total, c);
+    if (it >= items) continue;
+    int a = -1, rows = 0, first = 0;
+    if (i < used) {
+      a = c;
+      rows = min(kPlanTile, cnt - kPlanTile * (i - tb));
+      first = o + kPlanTile * (i - tb);
+    }
+    int32_t *rec = table + (size_t)i * kPlanRec;
+    if (q == 0) {
+      *reinterpret_cast<int4 *>(rec) = make_int4(a, rows, first, 0);
+    } else {
+      const int s0 = 4 * (q - 1);
+      if (s0 >= rows)
+        *reinterpret_cast<int4 *>(rec + 4 + s0) = make_int4(-1, -1, -1, -1);
+      else
+        for (int sl = rows; sl < s0 + 4; sl++) rec[4 + sl] = -1;
+    }
   }
 }
 
@@ -333,10 +376,22 @@ extern "C" bi_status bi_lora_plan(const int32_t *ids, int M, int n_adapters, voi
   if (!bi_aligned16(plan)) return BI_ERR_UNSUPPORTED_SHAPE;
   const int ncls = n_adapters + 1;
   const size_t smem = sizeof(int) * ((size_t)ncls * 4 + 2 + 64 + (size_t)bi::kPlanWarps * ncls);
-  if (n_adapters <= 31 && M <= bi::kPlanChunk)
-    bi::plan_small_kernel<<<1, bi::kPlanThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        ids, M, n_adapters, static_cast<int32_t *>(plan));
-  else
+  if (n_adapters <= 31 && M <= bi::kPlanChunk) {
+    cudaLaunchConfig_t cfg = {};
+    const unsigned ncta = (unsigned)std::max(1, (M + 511) / 512);
+    cfg.gridDim = dim3(ncta, 1, 1);
+    cfg.blockDim = dim3(32 * bi::kPlanSmallWarps, 1, 1);
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ncta;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int32_t *out = static_cast<int32_t *>(plan);
+    if (cudaLaunchKernelEx(&cfg, bi::plan_small_kernel, ids, M, n_adapters, out) != cudaSuccess) return BI_ERR_CUDA;
+  } else
     bi::plan_kernel<<<1, bi::kPlanThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
         ids, M, n_adapters, static_cast<int32_t *>(plan));
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
