@@ -209,18 +209,28 @@ def test_plan_matches_oracle(cfg4):
     check_plan_table(plan, np.concatenate([want_perm, invalid]).astype(np.int32), offs, 8)
 
 
-@pytest.mark.parametrize("M,n_ad", [(1, 1), (5, 3), (1000, 8), (4096, 8), (3000, 256), (0, 4),
-                                    (4097, 2), (12289, 8), (65536, 256)])
-def test_plan_shapes(M, n_ad):
+@pytest.mark.parametrize("M,n_ad,bad", [(1, 1, 0), (5, 3, 0), (1000, 8, 0), (4096, 8, 0), (3000, 256, 0),
+                                        (0, 4, 0), (4097, 2, 0), (12289, 8, 0), (65536, 256, 0), (4096, 31, 1),
+                                        (4096, 32, 1), (513, 64, 1), (20000, 31, 1), (100003, 5, 1),
+                                        (70001, 200, 1)])
+def test_plan_shapes(M, n_ad, bad):
+    """Every size path of the plan kernel (one chunk per warp or several,
+    at most 32 classes or more), with tokens outside every adapter where
+    `bad` is set (id -1 and id >= n_ad go to the last class)."""
     ids = synth.adapter_ids(M, n_ad, seed=M + n_ad)
+    if bad:
+        ids[::13] = -1
+        ids[7::29] = n_ad + 3
     plan = bi.lora_plan(dev(ids), n_ad).cpu().numpy() if M else None
     if M == 0:
         return
     want_perm, want_offs = oracle.segment(ids, n_ad)
+    invalid = np.nonzero((ids < 0) | (ids >= n_ad))[0]
+    full = np.concatenate([want_perm, invalid]).astype(np.int32)
     assert np.array_equal(plan[M:M + n_ad + 1], want_offs)
-    assert np.array_equal(plan[:M], want_perm)
+    assert np.array_equal(plan[:M], full)
     assert plan[M + n_ad + 1] == M
-    check_plan_table(plan, want_perm, plan[M:M + n_ad + 2], n_ad)
+    check_plan_table(plan, full, plan[M:M + n_ad + 2], n_ad)
 
 
 @pytest.mark.parametrize("r", [8, 16, 64])
