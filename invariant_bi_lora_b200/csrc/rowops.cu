@@ -225,6 +225,7 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   __shared__ float s_red[32];
   __shared__ float s_max, s_sum;
   __shared__ float s_maxs[16], s_sums[16];     // the cluster's values, pushed by their owners
+  __shared__ __align__(8) uint64_t s_bar[2];   // [0]: all C maxes landed, [1]: all C sums
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.C;
   const int q = (int)cluster.block_rank();
@@ -239,8 +240,19 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   // this lane's vectors: 4096*j + lane_id for j < nj
   const int nj = lane_id < nvec ? (nvec - 1 - lane_id) / kLsmT + 1 : 0;
 
-  // every CTA of the cluster has started once this arrive is matched; the
-  // wait comes before the first write into a peer's shared memory
+  // Each CTA pushes its max, then its sum, into slot q of every CTA with
+  // st.async; a CTA's barrier counts the 4 * C bytes that land in its own
+  // slots, so it waits for exactly the values it reads and no CTA waits for
+  // another's threads.  The barriers are initialised before the cluster
+  // arrive; every CTA has started (and initialised) once it is matched, and
+  // the wait comes before the first push.
+  if (tau == 0) {
+    mbar_init(&s_bar[0], 1);
+    mbar_init(&s_bar[1], 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(&s_bar[0], 4u * C);
+    mbar_arrive_expect_tx(&s_bar[1], 4u * C);
+  }
   cluster_arrive_relaxed();
 
   // ---- this lane's vectors -> its shared-memory slots: 16-byte cp.async
@@ -266,9 +278,8 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
   __syncthreads();
   cluster_wait();
   // push this CTA's max into slot q of every CTA of the cluster
-  if (tau < C) *cluster.map_shared_rank(&s_maxs[q], tau) = s_max;
-  cluster_arrive_release();
-  cluster_wait_acquire();
+  if (tau < C) st_async_f32(&s_maxs[q], &s_bar[0], (uint32_t)tau, s_max);
+  if (!mbar_wait_cluster(&s_bar[0], 0)) flag_error(p.status, BI_ERR_TIMEOUT);
   // row max over the cluster (exact in any order), from this CTA's own slots
   float rmax = s_maxs[0];
   for (int t = 1; t < C; t++) rmax = fmaxf(rmax, s_maxs[t]);
@@ -298,12 +309,11 @@ log_softmax_kernel(const __grid_constant__ LsmParams p) {
     if (tau == 0) s_sum = v;
   }
   __syncthreads();
-  // push this CTA's subtree value into slot q of every CTA; after the
-  // barrier nothing reads or writes a peer's memory, so no CTA waits for the
-  // others before it exits
-  if (tau < C) *cluster.map_shared_rank(&s_sums[q], tau) = s_sum;
-  cluster_arrive_release();
-  cluster_wait_acquire();
+  // push this CTA's subtree value into slot q of every CTA.  These are the
+  // last writes into a peer's memory, and a peer cannot pass its own wait
+  // before they land, so no CTA waits for the others before it exits.
+  if (tau < C) st_async_f32(&s_sums[q], &s_bar[1], (uint32_t)tau, s_sum);
+  if (!mbar_wait_cluster(&s_bar[1], 0)) flag_error(p.status, BI_ERR_TIMEOUT);
   // perfect tree over the C CTA subtrees (lanes 0..C-1, xor butterfly:
   // pairs, then pairs of pairs); every warp computes it from its own copy
   float v = (tau & 31) < C ? s_sums[tau & 31] : 0.0f;

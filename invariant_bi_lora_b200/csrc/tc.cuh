@@ -69,6 +69,39 @@ BI_DEV bool mbar_wait_for(uint64_t *bar, uint32_t parity, unsigned long long lim
   }
 }
 BI_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitLimitNs); }
+// The same with cluster-scope acquire: data that peers delivered with
+// st.async (counted on this barrier) is visible once the phase is seen.
+BI_DEV bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+BI_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; i++)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+// 4-byte store into CTA `rank`'s shared memory (the same offset as `local`
+// there), counted as 4 bytes of transaction on that CTA's barrier at the
+// offset of `local_bar`.
+BI_DEV void st_async_f32(float *local, uint64_t *local_bar, uint32_t rank, float v) {
+  uint32_t dst, bar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(smem_u32(local_bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(dst), "f"(v),
+               "r"(bar)
+               : "memory");
+}
 
 // ------------------------------------------------------------------ TMA
 // 2-D tile load into shared memory, completion counted on `bar` (bytes).
