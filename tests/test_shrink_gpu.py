@@ -275,3 +275,42 @@ def test_status_clean_after_shrink(cfg1):
     x, at = (dev_bf16(a) for a in cfg1)
     run_shrink(x, at, 8, "tree")
     assert bi.get_device_status() == 0
+
+
+@pytest.mark.parametrize("K,r", [(4096, 16), (2048, 16), (4096, 8), (2048, 8)])
+def test_large_ragged_batch(K, r):
+    """A batch of 4099 tokens (several waves of row tiles, a ragged last
+    tile, rows without an adapter): in modes TREE and UNSPLIT every row
+    must equal, bit for bit, the same row computed in a small batch, rows
+    without an adapter must be zero, and a ragged plain batch must match
+    too."""
+    M = 4099
+    d = synth.lora_inputs(M, K, r, n_adapters=5, seed=K + r)
+    x, at, ids = d["x"], d["at"], d["ids"].copy()
+    ids[::11] = -1
+    ids[3::17] = 9                         # out of range: no adapter
+    X, A = dev_bf16(x), dev_bf16(at)
+    plan = bi.lora_plan(dev(ids), 5)
+    got = {}
+    for mode, s in (("tree", 8), ("unsplit", 1), ("tree", 4)):
+        y = torch.full((M, r), 7.0, dtype=torch.float32, device="cuda")
+        bi.lora_shrink_segmented(X, A, plan, y, splits=s, mode=mode)
+        got[(mode, s)] = host_bits(y)
+    ref = got[("tree", 8)]
+    for k, v in got.items():
+        assert np.array_equal(v, ref), k
+    none = (ids < 0) | (ids >= 5)
+    assert np.all(ref.view(np.float32)[none] == 0.0)
+    for a in range(5):
+        sel = np.nonzero(ids == a)[0]
+        sel = np.concatenate([sel[:24], sel[-24:]])
+        y1 = host_bits(run_shrink(dev_bf16(x[sel]), dev_bf16(at[a]), 8, "tree"))
+        assert np.array_equal(ref[sel], y1), a
+    # plain (single adapter) batch with a ragged last tile
+    y = host_bits(run_shrink(X, dev_bf16(at[0]), 8, "tree"))
+    tail = np.arange(M - 21, M)
+    y1 = host_bits(run_shrink(dev_bf16(x[tail]), dev_bf16(at[0]), 8, "tree"))
+    assert np.array_equal(y[tail], y1)
+    exact, bound = oracle.shrink_exact(x[tail], at[0])
+    assert_tol(y[tail].view(np.float32), exact, bound)
+    assert bi.get_device_status() == 0
