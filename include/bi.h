@@ -172,7 +172,9 @@ bi_status bi_lora_fused(const void *x, const void *A, const void *B, const void 
 bi_status bi_lora_expand(const float *y, const void *B, float *out,
                          int M, int r, int N, int accumulate, bi_stream_t stream);
 
-/* Segmented expand: B bf16 [n_adapters][N][r]; plan from bi_lora_plan. */
+/* Segmented expand: B bf16 [n_adapters][N][r]; plan from bi_lora_plan  */
+/* (16-byte aligned, else BI_ERR_UNSUPPORTED_SHAPE).  A CTA reads its 64  */
+/* rows' adapter and token ids from one record of the plan's tile table. */
 bi_status bi_lora_expand_segmented(const float *y, const void *B, const void *plan,
                                    int n_adapters, float *out, int M, int r, int N,
                                    int accumulate, bi_stream_t stream);

@@ -89,65 +89,9 @@ BI_DEV float warp_max(float v) {
   return v;
 }
 
-// ----------------------------------------------------------------------
-// Row tiles of the multi-adapter (segmented) kernels.  A plan (see
-// bi_lora_plan) lists the tokens grouped by adapter: perm[offsets[a] ..
-// offsets[a+1]) are adapter a's tokens, a = n_ad being the tokens without
-// an adapter.  Tiles of `bm` rows never straddle two segments; tile t is
-// found by walking the segments.  offsets == nullptr: one segment, rows
-// 0..M-1 in order, adapter 0.
-// ----------------------------------------------------------------------
-struct TileInfo {
-  int adapter;     // -1: past the last tile; n_ad: the "no adapter" segment
-  int seg_begin;   // first perm position of the segment
-  int row0;        // first position of the tile inside the segment
-  int rows;        // rows in the tile (<= bm)
-};
-
-BI_DEV TileInfo resolve_tile(const int32_t *offsets, int n_ad, int M, int tile, int bm) {
-  TileInfo ti{-1, 0, 0, 0};
-  if (offsets == nullptr) {
-    if ((long)tile * bm < M) {
-      ti.adapter = 0;
-      ti.row0 = tile * bm;
-      ti.rows = min(bm, M - tile * bm);
-    }
-    return ti;
-  }
-  for (int a = 0; a <= n_ad; a++) {
-    const int b = offsets[a], e = offsets[a + 1];
-    const int nt = (e - b + bm - 1) / bm;
-    if (tile < nt) {
-      ti.adapter = a;
-      ti.seg_begin = b;
-      ti.row0 = tile * bm;
-      ti.rows = min(bm, e - b - tile * bm);
-      return ti;
-    }
-    tile -= nt;
-  }
-  return ti;
-}
-
-// resolve_tile for a whole CTA (every thread calls it): the n_ad + 2
-// segment starts are fetched by parallel loads into shared memory `s_off`
-// (room for kMaxAdapters + 2) and scanned there, so finding the tile costs
-// one memory round trip whatever its segment.  The result lands in *out
-// (shared) and is visible to every thread on return.
+// Largest adapter count of a plan (segment n_ad holds the tokens without
+// an adapter).
 constexpr int kMaxAdapters = 256;
-BI_DEV void resolve_tile_block(const int32_t *offsets, int n_ad, int M, int tile, int bm, int32_t *s_off,
-                               TileInfo *out) {
-  if (offsets)
-    for (int t = threadIdx.x; t < n_ad + 2; t += blockDim.x) s_off[t] = offsets[t];
-  __syncthreads();
-  if (threadIdx.x == 0) *out = resolve_tile(offsets ? s_off : nullptr, n_ad, M, tile, bm);
-  __syncthreads();
-}
-
-// Token index of position `pos` of a tile (identity without a plan).
-BI_DEV int tile_row(const int32_t *perm, const TileInfo &ti, int local) {
-  return perm ? perm[ti.seg_begin + ti.row0 + local] : ti.row0 + local;
-}
 
 // ----------------------------------------------------------------------
 // Plan layout (int32 words), written by bi_lora_plan:
