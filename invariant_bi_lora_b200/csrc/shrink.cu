@@ -290,6 +290,20 @@ BI_DEV void fused_expand(const ShrinkParams &p, const float *yfull, const int32_
   }
 }
 
+// Mode TREE: the exchange barrier of this CTA counts the bytes its peers
+// push into its slots (st.async), so a rank waits for exactly the shares it
+// adds and never for its peers' threads.  Initialised, with its expected
+// bytes, by one thread before the cluster arrive that every CTA makes on
+// entry (the fence makes the initialisation visible to the cluster).
+BI_DEV void exchange_init(const ShrinkParams &p, int bm, int split, uint64_t *xbar) {
+  const uint32_t E = (uint32_t)bm * p.r;
+  const uint32_t S = p.splits;
+  const uint32_t bytes = p.gather0 ? (split == 0 ? (S - 1) * E * 4 : 0u) : (S - 1) * (E / S) * 4;
+  mbar_init(xbar, 1);
+  mbar_fence_init();
+  mbar_arrive_expect_tx(xbar, bytes);
+}
+
 // The G group values of a row tile (part [G][bm][r], in shared memory,
 // written and visible to the CTA) -> the tile's y rows: the perfect tree over
 // the groups, then the cross-split combine of the mode.  Every thread of the
@@ -299,7 +313,7 @@ BI_DEV void fused_expand(const ShrinkParams &p, const float *yfull, const int32_
 // With p.fuse, the final y values also go to yfull in every CTA of the tile
 // (all-gather through distributed shared memory), and the tile's expand
 // follows; y itself is written only when p.y is set.
-BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const int32_t *s_rows,
+BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, uint64_t *xbar, const int32_t *s_rows,
                         int rows, int bm, int split, int adapter) {
   const int E = bm * p.r;
   const int r_sh = (p.r & (p.r - 1)) == 0 ? __ffs(p.r) - 1 : -1;
@@ -335,13 +349,14 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
 
   // ---- mode TREE: the splits CTAs of this tile form one cluster; rank q
   // holds the subtree of leaves [q*lc, (q+1)*lc).  The tile's E elements
-  // are cut into S shares; rank q finishes share q.  Before one cluster
-  // barrier every rank stores share t of its partial into rank t's slot
-  // [q] through distributed shared memory (a reduce-scatter by pushes);
-  // after it (release / acquire) each rank adds the S values of its share
-  // by the perfect tree over the ranks, from its own shared memory, and
-  // writes y.  Nothing reads a peer's memory after the barrier, so one
-  // barrier is enough, and every SM receives only (S-1)/S of one partial.
+  // are cut into S shares; rank q finishes share q.  Every rank stores share
+  // t of its partial into rank t's slot [q] by st.async (a reduce-scatter by
+  // pushes), counted on rank t's exchange barrier; once its own barrier has
+  // seen all S-1 shares land, each rank adds the S values of its share by
+  // the perfect tree over the ranks, from its own shared memory, and writes
+  // y.  Nothing reads a peer's memory, and every SM receives only (S-1)/S of
+  // one partial.  A rank cannot finish before every share pushed to it has
+  // landed, so no rank waits for its peers before it exits.
   cg::cluster_group cluster = cg::this_cluster();
   const int S = p.splits;
   // the relaxed arrive each CTA made on entry: once this wait returns,
@@ -358,13 +373,12 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
     // slots [S-1][E]; after the barrier rank 0 alone adds and writes y
     float *gslots = slots;
     if (split != 0) {
-      float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(gslots, 0) + (size_t)(split - 1) * E);
       const float4 *src = reinterpret_cast<const float4 *>(part);
-      for (int e4 = threadIdx.x; e4 < E / 4; e4 += blockDim.x) dst[e4] = src[e4];
+      for (int e4 = threadIdx.x; e4 < E / 4; e4 += blockDim.x)
+        st_async_v4(gslots + (size_t)(split - 1) * E + 4 * e4, xbar, 0u, src[e4]);
     }
-    cluster_arrive_release();
-    cluster_wait_acquire();
     if (split == 0) {
+      if (!mbar_wait_cluster(xbar, 0)) flag_error(p.status, BI_ERR_TIMEOUT);
       for (int e = threadIdx.x; e < valid_E; e += blockDim.x) {
         float v[kMaxSplits];
         v[0] = part[e];
@@ -382,12 +396,11 @@ BI_DEV void finish_tile(const ShrinkParams &p, float *part, float *slots, const 
     const int share = E / S;                         // E = 16 * mt * r, a multiple of 128
     for (int t = 0; t < S; t++) {
       if (t == split) continue;
-      float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(slots, t) + (size_t)split * share);
       const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * share);
-      for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x) dst[i4] = src[i4];
+      for (int i4 = threadIdx.x; i4 < share / 4; i4 += blockDim.x)
+        st_async_v4(slots + (size_t)split * share + 4 * i4, xbar, (uint32_t)t, src[i4]);
     }
-    cluster_arrive_release();
-    cluster_wait_acquire();
+    if (!mbar_wait_cluster(xbar, 0)) flag_error(p.status, BI_ERR_TIMEOUT);
     for (int i = threadIdx.x; i < share; i += blockDim.x) {
       const int e = split * share + i;
       if (e >= valid_E) break;
@@ -423,19 +436,21 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   float *part = reinterpret_cast<float *>(smem_f4);     // [G][BM][r]
   __shared__ int32_t s_rows[kMaxBM];                    // token row of each tile row
   __shared__ int s_info[2];
+  __shared__ __align__(8) uint64_t s_xbar;              // mode TREE exchange barrier
 
   const int bm = 16 * p.mtiles;
   const int split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
+  const bool clustered = p.mode == BI_SHRINK_TREE && p.splits > 1;
 
   if (warp == 0) tile_record(p, bm, blockIdx.y, lane, s_rows, s_info);
+  if (clustered && threadIdx.x == 32 % blockDim.x) exchange_init(p, bm, split, &s_xbar);
   __syncthreads();
   struct { int adapter, rows; } ti = {s_info[0], s_info[1]};
   // mode TREE: say "started" to the cluster now; finish_tile waits for the
   // others before it writes into their shared memory.  The exits below are
   // uniform across the cluster (every split sees the same tile) and wait too.
-  const bool clustered = p.mode == BI_SHRINK_TREE && p.splits > 1;
   if (clustered) cluster_arrive_relaxed();
   if (ti.adapter < 0) {
     if (clustered) cluster_wait();
@@ -645,7 +660,7 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
   }
   __syncthreads();
   float *slots = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(smem_f4) + p.g_offset);
-  finish_tile(p, part, slots, s_rows, ti.rows, bm, split, ti.adapter);
+  finish_tile(p, part, slots, &s_xbar, s_rows, ti.rows, bm, split, ti.adapter);
 }
 
 // ----------------------------------------------------------------------
@@ -658,7 +673,7 @@ shrink_kernel(const __grid_constant__ ShrinkParams p) {
 // multiplying as soon as their rows are in.  Used when the slice fits:
 // lc <= 16 leaves per split (e.g. K = 4096 at splits >= 4).
 //
-// Shared memory: [0, 64) mbarriers (m-tiles 0..3, A = 4); [64, 320) token
+// Shared memory: [0, 64) mbarriers (m-tiles 0..3, A = 4, TREE exchange = 5); [64, 320) token
 // rows; [320, 328) adapter and rows; x rows at x_off (row stride rowbytes);
 // A rows at a_offset; the group values at part_off (they may overlay the x
 // rows, which are dead by then); the TREE exchange slots at g_offset.
@@ -677,7 +692,7 @@ shrink_bulk_kernel(const __grid_constant__ ShrinkParams p) {
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   int32_t *s_rows = reinterpret_cast<int32_t *>(smem + 64);
   int *s_info = reinterpret_cast<int *>(smem + 320);
-  constexpr int kABar = 4;
+  constexpr int kABar = 4, kXBar = 5;           // A-slice barrier, TREE exchange barrier
 
   const int bm = 16 * p.mtiles;
   const int split = blockIdx.x;
@@ -691,6 +706,7 @@ shrink_bulk_kernel(const __grid_constant__ ShrinkParams p) {
 #pragma unroll
     for (int i = 0; i <= kABar; i++) mbar_init(&bars[i], 1);
     mbar_fence_init();
+    if (p.mode == BI_SHRINK_TREE && p.splits > 1) exchange_init(p, bm, split, &bars[kXBar]);
   }
   __syncthreads();
   const int adapter = s_info[0], rows = s_info[1];
@@ -830,7 +846,7 @@ shrink_bulk_kernel(const __grid_constant__ ShrinkParams p) {
   }
   __syncthreads();
   float *slots = reinterpret_cast<float *>(smem + p.g_offset);
-  finish_tile(p, part, slots, s_rows, rows, bm, split, adapter);
+  finish_tile(p, part, slots, &bars[kXBar], s_rows, rows, bm, split, adapter);
 }
 
 // ----------------------------------------------------------------------

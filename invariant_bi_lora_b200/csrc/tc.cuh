@@ -91,6 +91,18 @@ BI_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned long long
     if (global_ns() - t0 > limit_ns) return false;
   }
 }
+// 16-byte store into CTA `rank`'s shared memory (the same offset as `local`
+// there, 16-byte aligned), counted as 16 bytes of transaction on that CTA's
+// barrier at the offset of `local_bar`.
+BI_DEV void st_async_v4(float *local, uint64_t *local_bar, uint32_t rank, float4 v) {
+  uint32_t dst, bar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(smem_u32(local_bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+               : "memory");
+}
 // 4-byte store into CTA `rank`'s shared memory (the same offset as `local`
 // there), counted as 4 bytes of transaction on that CTA's barrier at the
 // offset of `local_bar`.
