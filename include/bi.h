@@ -236,6 +236,22 @@ bi_status bi_gemm_tree(const void *A, const void *W, float *C, int M, int N, int
 bi_status bi_tree_combine(const float *partials, float *out, int s, size_t count,
                           bi_stream_t stream);
 
+/* Cross-GPU combine [TBIK Abstract: the inter-GPU reduction follows the  */
+/* same tree]: out[i] = tree(partials[0][i], ..., partials[s-1][i]) for   */
+/* i in [begin, begin + count), the same tree as bi_tree_combine.         */
+/* partials: a HOST array of s device pointers, each to an fp32 [total]   */
+/* partial that this device can load from -- its own memory or a peer     */
+/* GPU's (peer access or CUDA IPC / symmetric memory); the kernel reads    */
+/* them with plain loads (no multicast) and writes out[begin ..) of its    */
+/* own memory.  A rank that combines only its share [begin, begin+count)  */
+/* gives a reduce-scatter; every rank combining everything, an all-reduce */
+/* in the canonical order.  The caller orders the partials' writes before */
+/* the call on every GPU (a barrier) and keeps them alive until the call  */
+/* has finished on every GPU.  s in [1, 64]; begin and count multiples of */
+/* 4; every pointer 16-byte aligned, else BI_ERR_UNSUPPORTED_SHAPE.       */
+bi_status bi_tree_combine_peers(const float *const *partials, int s, float *out, size_t begin,
+                                size_t count, bi_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* Batch-invariant row operations, one CTA (or one cluster) per row, so  */
 /* row i's bits never depend on how many rows there are.  The row sum S */

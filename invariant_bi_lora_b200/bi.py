@@ -48,6 +48,7 @@ _SIGS = {
     "bi_gemm_tree_partials": (I, [P, P, P, I, I, I, I, P]),
     "bi_gemm_tree": (I, [P, P, P, I, I, I, I, P, Z, P]),
     "bi_tree_combine": (I, [P, P, I, Z, P]),
+    "bi_tree_combine_peers": (I, [ctypes.POINTER(ctypes.c_void_p), I, P, Z, Z, P]),
     "bi_rmsnorm": (I, [P, P, P, I, I, F, P]),
     "bi_log_softmax": (I, [P, P, I, I, P]),
     "bi_mean": (I, [P, P, I, I, P]),
@@ -307,6 +308,19 @@ def tree_combine(partials, out, stream=None):
     if partials.numel() != s * out.numel():
         raise ValueError("shape mismatch")
     _call("bi_tree_combine", _ptr(partials), _ptr(out), s, out.numel(), _stream(stream))
+    return out
+
+
+def tree_combine_peers(ptrs, out, begin=0, count=None, stream=None):
+    """out[begin:begin+count] = canonical tree over the partials behind the
+    device pointers `ptrs` (ints; each partial fp32 with out's numel, in this
+    GPU's memory or a peer's), read with plain loads in one kernel."""
+    _check(out, "out", torch.float32)
+    count = out.numel() - begin if count is None else count
+    if begin < 0 or count < 0 or begin + count > out.numel():
+        raise ValueError("range outside out")
+    arr = (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(int(q)) for q in ptrs])
+    _call("bi_tree_combine_peers", arr, len(ptrs), _ptr(out), begin, count, _stream(stream))
     return out
 
 

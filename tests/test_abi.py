@@ -73,6 +73,16 @@ def test_other_rejects(libbi):
     assert libbi.bi_mean(FAKE, FAKE, -1, 8, None) == 1
     assert libbi.bi_tree_combine(FAKE, FAKE, 0, 16, None) == 1
     assert libbi.bi_tree_combine(FAKE, FAKE, 65, 16, None) == 1
+    ptrs2 = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert libbi.bi_tree_combine_peers(ptrs2, 0, FAKE, 0, 16, None) == 1            # s < 1
+    assert libbi.bi_tree_combine_peers(ptrs2, 65, FAKE, 0, 16, None) == 1           # s > 64
+    assert libbi.bi_tree_combine_peers(None, 2, FAKE, 0, 16, None) == 1             # no pointer array
+    assert libbi.bi_tree_combine_peers(ptrs2, 2, FAKE, 2, 16, None) == 2            # begin not a multiple of 4
+    bad = (ctypes.c_void_p * 2)(FAKE, ctypes.c_void_p(0x10004))
+    assert libbi.bi_tree_combine_peers(bad, 2, FAKE, 0, 16, None) == 2              # a partial misaligned
+    nul = (ctypes.c_void_p * 2)(FAKE, None)
+    assert libbi.bi_tree_combine_peers(nul, 2, FAKE, 0, 16, None) == 1              # a null partial
+    assert libbi.bi_tree_combine_peers(ptrs2, 2, FAKE, 0, 0, None) == 0             # empty range: no-op
     assert libbi.bi_math_spec(FAKE, FAKE, 16, 4, None) == 1
     assert libbi.bi_selftest_bounded_wait(0, None) == 1
 

@@ -2,7 +2,8 @@
 
 - max_over_ranks: the bench's device-time reduction (every rank gets the
   elementwise maximum).
-- tree_gemm_tp: the tensor-parallel exchange of the tree GEMM ("Deterministic
+- tree_gemm_tp and tree_gemm_tp_peers: the tensor-parallel exchange of the
+  tree GEMM, by all-gather and by peer loads ("Deterministic
   Inference across Tensor Parallel Sizes That Eliminates Training-Inference
   Mismatch", Abstract).  Each rank computes the subtree over its own K range,
   the partials are gathered in rank order and the top levels are added.  The
@@ -22,7 +23,7 @@ import torch.multiprocessing as mp
 
 import oracle
 from invariant_bi_lora_b200 import synth
-from invariant_bi_lora_b200.tp import LEAF, max_over_ranks, shard_k_range, tree_gemm_tp
+from invariant_bi_lora_b200.tp import LEAF, max_over_ranks, shard_k_range, tree_gemm_tp, tree_gemm_tp_peers
 
 M, N, K = 24, 16, 2048          # 8 leaves of 256
 
@@ -72,6 +73,30 @@ def _worker(rank, world, port, result_dir):
         C = torch.empty(M, N, dtype=torch.float32)
         tree_gemm_tp(a_loc, w_loc, C, partial_fn=partial_fn, combine_fn=combine_fn)
         np.save(os.path.join(result_dir, f"c{rank}.npy"), _bits(C))
+
+        # the peer-load exchange: the partial goes into this rank's shared
+        # buffer; "peer loads" are stood in for by gathering the buffers
+        # (on CPU there is no peer memory), after the first barrier
+        class Peers:
+            buf = torch.full((M, N), 7.0, dtype=torch.float32)
+            ptrs = list(range(world))
+        events = []
+
+        def combine_peers_fn(peers, out):
+            got = [torch.empty_like(peers.buf) for _ in range(world)]
+            dist.all_gather(got, peers.buf)
+            events.append("combine")
+            out.copy_(torch.from_numpy(oracle.tree_combine(torch.stack(got).numpy())))
+
+        def barrier_fn(group):
+            events.append("barrier")
+            dist.barrier(group=group)
+
+        C2 = torch.empty(M, N, dtype=torch.float32)
+        tree_gemm_tp_peers(a_loc, w_loc, C2, Peers(), partial_fn=partial_fn, combine_peers_fn=combine_peers_fn,
+                           barrier_fn=barrier_fn)
+        assert events == ["barrier", "combine", "barrier"], events
+        np.save(os.path.join(result_dir, f"p{rank}.npy"), _bits(C2))
     finally:
         dist.destroy_process_group()
 
@@ -152,3 +177,4 @@ def test_tp_tree_gemm_ranks(tmp_path, world):
     for r in range(world):
         got = np.load(tmp_path / f"c{r}.npy")
         assert np.array_equal(got, want), r
+        assert np.array_equal(np.load(tmp_path / f"p{r}.npy"), want), r
