@@ -25,8 +25,8 @@
 //    the counts sit in a per-warp shared-memory row that the first lane of
 //    each class group advances.
 //  * Bases: pass 1 counts; every warp pushes its row of class counts into
-//    every CTA's [warp][class] table, and after one cluster barrier each
-//    warp scans the whole table itself (its class bases in the warps before
+//    every CTA's [warp][class] table by st.async, counted on that CTA's
+//    mbarrier, and once its own table is complete each warp scans it itself (its class bases in the warps before
 //    it, the class totals; a shuffle scan over the classes gives the
 //    segment starts and the table bases).  Pass 2 ranks again from those
 //    bases and scatters (one chunk per warp, the common case, keeps pass 1's
@@ -38,7 +38,6 @@
 #include "tc.cuh"
 
 #include <algorithm>
-#include <cooperative_groups.h>
 
 namespace bi {
 
@@ -94,9 +93,7 @@ BI_DEV int plan_bump(int *cnt, int cls, unsigned same, unsigned lt_mask) {
 // wide adds cnt[W][ncls], s_off[ncls + 1], s_tb[ncls + 1].
 template <bool WIDE>
 __global__ void __launch_bounds__(512)
-plan_kernel(const int32_t *__restrict__ ids, int M, int n_ad, int cpw, int32_t *__restrict__ plan) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
+plan_kernel(const int32_t *__restrict__ ids, int M, int n_ad, int cpw, int32_t *__restrict__ plan, unsigned *status) {
   extern __shared__ int plan_smem[];
   const int ncls = n_ad + 1, ncta = gridDim.x, W = blockDim.x >> 5;   // the grid is one cluster
   const int lane = threadIdx.x & 31, lw = threadIdx.x >> 5;
@@ -111,8 +108,14 @@ plan_kernel(const int32_t *__restrict__ ids, int M, int n_ad, int cpw, int32_t *
   int32_t *offsets = plan + M;
   int32_t *table = plan + plan_table_word(M, n_ad);
   const int ntiles = (int)plan_tiles(M, n_ad);
-  // every CTA has started once this arrive is matched; the wait comes
-  // before the first write into a peer's shared memory
+  // every CTA has started (and initialised its table barrier) once this
+  // arrive is matched; the wait comes before the first push into a peer
+  __shared__ __align__(8) uint64_t s_tbar;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_tbar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(&s_tbar, 4u * (uint32_t)nw * (uint32_t)ncp);
+  }
   cluster_arrive_relaxed();
   // start the output's address translation while the ids are in flight
   if (warp == 0 && lane == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(plan));
@@ -151,19 +154,18 @@ plan_kernel(const int32_t *__restrict__ ids, int M, int n_ad, int cpw, int32_t *
     if (k == 0) run0 = run;
   }
 
-  // ---- counts into every CTA's table, one cluster barrier
+  // ---- counts into every CTA's table (nw * ncp words land in each)
   cluster_wait();
   if (WIDE) {
     for (int c = lane; c < ncls; c += 32) {
       const int v = cnt[c];
-      for (int r = 0; r < ncta; r++) *cluster.map_shared_rank(&tbl[warp * ncp + c], r) = v;
+      for (int r = 0; r < ncta; r++) st_async_u32(&tbl[warp * ncp + c], &s_tbar, (uint32_t)r, (uint32_t)v);
     }
   } else {
     const int v = lane < ncls ? run : 0;
-    for (int r = 0; r < ncta; r++) *cluster.map_shared_rank(&tbl[warp * ncp + lane], r) = v;
+    for (int r = 0; r < ncta; r++) st_async_u32(&tbl[warp * ncp + lane], &s_tbar, (uint32_t)r, (uint32_t)v);
   }
-  cluster_arrive_release();
-  cluster_wait_acquire();
+  if (!mbar_wait_cluster(&s_tbar, 0)) flag_error(status, BI_ERR_TIMEOUT);
 
   // ---- bases: this warp's start inside each class, segment starts, table bases
   int before = 0, total = 0, off = 0, tbase = 0, used = 0;   // narrow: lane c's class
@@ -331,8 +333,9 @@ extern "C" bi_status bi_lora_plan(const int32_t *ids, int M, int n_adapters, voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int32_t *out = static_cast<int32_t *>(plan);
-  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, bi::plan_kernel<true>, ids, M, n_adapters, cpw, out)
-                             : cudaLaunchKernelEx(&cfg, bi::plan_kernel<false>, ids, M, n_adapters, cpw, out);
+  unsigned *status = bi::status_word();
+  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, bi::plan_kernel<true>, ids, M, n_adapters, cpw, out, status)
+                             : cudaLaunchKernelEx(&cfg, bi::plan_kernel<false>, ids, M, n_adapters, cpw, out, status);
   if (e != cudaSuccess) return BI_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

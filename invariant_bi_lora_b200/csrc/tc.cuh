@@ -91,6 +91,15 @@ BI_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned long long
     if (global_ns() - t0 > limit_ns) return false;
   }
 }
+// 4-byte integer store into CTA `rank`'s shared memory, counted like st_async_f32.
+BI_DEV void st_async_u32(void *local, uint64_t *local_bar, uint32_t rank, uint32_t v) {
+  uint32_t dst, bar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(smem_u32(local_bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst), "r"(v),
+               "r"(bar)
+               : "memory");
+}
 // 16-byte store into CTA `rank`'s shared memory (the same offset as `local`
 // there, 16-byte aligned), counted as 16 bytes of transaction on that CTA's
 // barrier at the offset of `local_bar`.
