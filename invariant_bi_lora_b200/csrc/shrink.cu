@@ -17,7 +17,8 @@
 // folds its group's leaves in post order in registers, the G group values
 // meet in shared memory (perfect tree), and in mode TREE the `splits` CTAs
 // of a row tile -- one thread-block cluster -- meet through distributed
-// shared memory (a reduce-scatter of pushes, one cluster barrier), perfect
+// shared memory (a reduce-scatter of st.async pushes, each rank waiting on
+// its own barrier for the shares it adds), perfect
 // tree again.  Every level is a level
 // of the one canonical tree over the K/64 leaves, so the bits cannot depend
 // on how the work was cut.
