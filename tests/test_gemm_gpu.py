@@ -24,7 +24,8 @@ def run_gemm(a, w, bf16_out=False):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 4096, 4096), (64, 512, 4096), (130, 272, 64),
-                                   (256, 4096, 192), (1024, 4096, 4096), (129, 16, 128), (300, 1040, 1024)])
+                                   (256, 4096, 192), (1024, 4096, 4096), (129, 16, 128), (300, 1040, 1024),
+                                   (2200, 512, 1024), (4096, 256, 256)])
 def test_gemm_tolerance(M, N, K):
     a, w = synth.gemm_inputs(M, N, K, seed=M + N + K)
     C = run_gemm(dev_bf16(a), dev_bf16(w)).cpu().numpy()
@@ -64,15 +65,17 @@ def test_gemm_bf16_output():
 def test_gemm_batch_invariance(N):
     """Rows of the M=1 result == the same rows at M = 16 ... 4096 (K=4096),
     wherever they sit in a tile; the M values cross the tile-width changes
-    (128 x 32 up to M = 128, 128 x 64 up to 512, 128 x 256 above)."""
+    (128 x 32 up to M = 128, 128 x 64 up to 512, 128 x 256 above) and end
+    with ragged last tiles."""
     K = 4096
     big_a, w = synth.gemm_inputs(4096, N, K, seed=7)
     W = dev_bf16(w)
     probe = big_a[:8]
     ref = np.stack([host_bits(run_gemm(dev_bf16(probe[i:i + 1]), W))[0] for i in range(8)])
-    for M in (16, 64, 128, 129, 256, 512, 513, 1024, 4096):
+    for M in (16, 64, 128, 129, 256, 512, 513, 1024, 2047, 2048, 2200, 4096):
         a = big_a[:M].copy()
-        positions = sorted({0, M - 1, min(127, M - 1), min(128, M - 1), M // 2, max(0, M - 8)})
+        positions = sorted({0, M - 1, min(127, M - 1), min(128, M - 1), min(255, M - 1), min(256, M - 1), M // 2,
+                            max(0, M - 8), max(0, M - 130)})
         for j, pos in enumerate(positions):
             a[pos] = probe[j % 8]
         C = host_bits(run_gemm(dev_bf16(a), W))
@@ -101,7 +104,8 @@ def test_gemm_rejects():
             dev_bf16(synth.normal_bf16((16, 64), 1.0, seed=1)), C)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (64, 512, 1024), (300, 1040, 1024), (1024, 4096, 4096)])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (64, 512, 1024), (300, 1040, 1024), (1024, 4096, 4096),
+                                   (2200, 1024, 512)])
 def test_addmm(M, N, K):
     """torch.addmm ("Batch Invariant Ops", Highlighted Details): within
     tolerance of the oracle's exact bias + A.W^T, and bitwise the GEMM's fp32
