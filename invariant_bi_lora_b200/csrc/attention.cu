@@ -23,12 +23,13 @@
 // flops, so the work runs on the CUDA cores in exactly this order (the CPU
 // oracle reproduces it bit for bit) and is bound by the KV read.
 //
-// Kernel 1 (one CTA per chunk, kv head, sequence; 256 threads): the chunk's
-// V rows (contiguous, up to 128 KB at D = 256) are requested by one bulk
-// copy into shared memory at entry, while every lane loads one key row into
-// registers and folds its scores; the chunk partials (m_c, l_c,
-// o_c) of the G query heads that share the kv head go to the caller's
-// workspace.  Kernel 2 (one CTA per query head and sequence): the combine.
+// Kernel 1 (one CTA per chunk, kv head, sequence; 256 threads): every lane
+// loads one key row into registers and folds its scores; the PV sums read
+// V straight from global memory (a warp reads 128 contiguous bytes of one V
+// row per slot), so a CTA needs ~18 KB of shared memory and three share an
+// SM; the chunk partials (m_c, l_c, o_c) of the G query heads that share
+// the kv head go to the caller's workspace.  Kernel 2 (one CTA per query
+// head and sequence): the combine.
 #include "bimath.cuh"
 #include "tc.cuh"
 
@@ -64,21 +65,20 @@ BI_DEV float counter_fold(int i, float x, float (&lv)[LEVELS > 0 ? LEVELS : 1]) 
   return x;
 }
 
+// Three CTAs per SM where the registers allow it without spilling (G * D <=
+// 512: the common D = 128, four query heads per kv head), else two.
 template <int D, int G>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__global__ void __launch_bounds__(kAttnThreads, G * D >= 1024 ? 2 : 3)
 attn_chunk_kernel(const __grid_constant__ AttnParams p) {
   constexpr int QT = 2 * kAttnThreads / D;          // threads per output column pair
   constexpr int SLOTS = kAttnChunk / QT;            // slots per thread in the PV sum
   constexpr int LV = SLOTS >= 128 ? 7 : SLOTS >= 64 ? 6 : 5;
   constexpr int GP = G >= 4 ? G : 4;                // p row padded to a float4
-  extern __shared__ __align__(128) uint8_t attn_smem[];
-  uint16_t *s_v = reinterpret_cast<uint16_t *>(attn_smem);            // [256][D] bf16
   __shared__ float s_q[G][D];
   __shared__ float s_p[G][kAttnChunk];             // scores
   __shared__ __align__(16) float s_pt[kAttnChunk][GP];   // p, [slot][head]
   __shared__ float s_red[G][8];
   __shared__ float s_half[G][QT][D];
-  __shared__ __align__(8) uint64_t s_bar;
 
   const int c = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int L = max(0, min(p.lens[b], p.Lmax));      // a length past Lmax reads nothing beyond it
@@ -88,15 +88,6 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t kvbase = (((size_t)b * p.Hkv + hk) * p.Lmax + j0) * D;
 
-  // the chunk's V rows (contiguous) go to shared memory by one bulk copy,
-  // in flight while the scores are computed
-  if (tid == 0) {
-    mbar_init(&s_bar, 1);
-    mbar_fence_init();
-    const uint32_t bytes = (uint32_t)nj * D * 2;
-    mbar_arrive_expect_tx(&s_bar, bytes);
-    bulk_load(s_v, p.v + kvbase, bytes, &s_bar);
-  }
   for (int e = tid; e < G * D; e += kAttnThreads) {
     const int i = e / D, d = e % D;
     s_q[i][d] = __uint_as_float((uint32_t)p.q[((size_t)b * p.Hq + hk * G + i) * D + d] << 16);
@@ -180,8 +171,6 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
     const float lw = warp_tree_sum(pv[i]);
     if (lane == 0) s_red[i][warp] = lw;
   }
-  const bool v_ok = mbar_wait(&s_bar, 0);           // the V rows
-  if (!v_ok) flag_error(p.status, BI_ERR_TIMEOUT);
   __syncthreads();
   float l_i[G];
 #pragma unroll
@@ -198,14 +187,28 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
 
   // ---- o_d: thread (part qt, columns 2dp and 2dp + 1) folds slots
   // [qt*SLOTS, +SLOTS) (a subtree) with the binary counter; one vector load
-  // gives every head's p of a slot; the QT subtrees meet in order
+  // gives every head's p of a slot; the QT subtrees meet in order.  V comes
+  // straight from global memory: a warp's 32 threads read 128 contiguous
+  // bytes of one V row per slot, eight slots' loads in flight ahead.
   const int dp = tid % (D / 2), qt = tid / (D / 2);
   float acc[G][2];
   float lv[G][2][LV];
+  const uint32_t *vcol = reinterpret_cast<const uint32_t *>(p.v + kvbase) + dp;   // V[j][2dp, 2dp+1]
+  constexpr int VPF = 8;
+  uint32_t vbuf[VPF];
+#pragma unroll
+  for (int s = 0; s < VPF; s++) {
+    const int j = qt * SLOTS + s;
+    vbuf[s] = j < nj ? __ldg(vcol + (size_t)j * (D / 2)) : 0u;
+  }
 #pragma unroll
   for (int s = 0; s < SLOTS; s++) {
     const int j = qt * SLOTS + s;
-    const uint32_t vw = *reinterpret_cast<const uint32_t *>(&s_v[j * D + 2 * dp]);
+    const uint32_t vw = vbuf[s % VPF];
+    if (s + VPF < SLOTS) {
+      const int jn = j + VPF;
+      vbuf[s % VPF] = jn < nj ? __ldg(vcol + (size_t)jn * (D / 2)) : 0u;
+    }
     const float v0 = j < nj ? bf16lo(vw) : 0.0f, v1 = j < nj ? bf16hi(vw) : 0.0f;
     float pj[GP];
 #pragma unroll
@@ -294,10 +297,7 @@ attn_combine_kernel(const __grid_constant__ AttnParams p) {
 template <int D, int G>
 static cudaError_t attn_chunk_launch(const AttnParams &p, cudaStream_t s) {
   const dim3 g1(p.max_chunks, p.Hkv, p.B);
-  constexpr size_t smem = (size_t)kAttnChunk * D * 2;          // the chunk's V rows
-  cudaError_t e = cudaFuncSetAttribute(attn_chunk_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  attn_chunk_kernel<D, G><<<g1, kAttnThreads, smem, s>>>(p);
+  attn_chunk_kernel<D, G><<<g1, kAttnThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
