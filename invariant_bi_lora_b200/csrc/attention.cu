@@ -26,7 +26,7 @@
 // Kernel 1 (one CTA per chunk, kv head, sequence; 256 threads): every lane
 // loads one key row into registers and folds its scores; the PV sums read
 // V straight from global memory (a warp reads 128 contiguous bytes of one V
-// row per slot), so a CTA needs ~18 KB of shared memory and three share an
+// row per slot), so a CTA needs ~18 KB of shared memory and four share an
 // SM; the chunk partials (m_c, l_c, o_c) of the G query heads that share
 // the kv head go to the caller's workspace.  Kernel 2 (one CTA per query
 // head and sequence): the combine.
@@ -65,10 +65,10 @@ BI_DEV float counter_fold(int i, float x, float (&lv)[LEVELS > 0 ? LEVELS : 1]) 
   return x;
 }
 
-// Three CTAs per SM where the registers allow it without spilling (G * D <=
-// 512: the common D = 128, four query heads per kv head), else two.
+// Four CTAs per SM (64 registers) where that costs no spill (G * D <= 512:
+// the common D = 128 with up to four query heads per kv head), else two.
 template <int D, int G>
-__global__ void __launch_bounds__(kAttnThreads, G * D >= 1024 ? 2 : 3)
+__global__ void __launch_bounds__(kAttnThreads, G * D >= 1024 ? 2 : 4)
 attn_chunk_kernel(const __grid_constant__ AttnParams p) {
   constexpr int QT = 2 * kAttnThreads / D;          // threads per output column pair
   constexpr int SLOTS = kAttnChunk / QT;            // slots per thread in the PV sum
