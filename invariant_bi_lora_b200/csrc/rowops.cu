@@ -125,6 +125,7 @@ rmsnorm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
 // (slot, warp) values in lane order by a perfect tree in one warp.
 // ======================================================================
 constexpr int kLaneT = 1024;
+constexpr int kMeanClusterRows = 128;        // up to this many rows: mean_cluster_kernel (measured crossover)
 constexpr int kMeanThreads = 256;
 
 __global__ void __launch_bounds__(kMeanThreads)
@@ -164,6 +165,73 @@ mean_kernel(const float *__restrict__ x, float *__restrict__ out, int n) {
     const float q = warp_tree_sum(s_grp[lane]);
     if (u == 0) out[row] = __fdiv_rn(q, (float)n);
   }
+}
+
+// Few rows: one cluster of C CTAs per row, CTA q owning the contiguous lanes
+// [q * 1024/C, (q+1) * 1024/C) -- a subtree of the 1024-lane tree, so the
+// bits are mean_kernel's.  Each CTA folds its lanes' chains (eight vector
+// loads in flight per lane) and its 32-lane groups, and pushes its value
+// into slot q of rank 0 by st.async; rank 0 adds the C values by the top
+// levels of the tree.  No CTA waits for another's threads.
+template <int C>
+__global__ void __launch_bounds__(kLaneT / C)
+mean_cluster_kernel(const float *__restrict__ x, float *__restrict__ out, int n, unsigned *status) {
+  constexpr int T = kLaneT / C, NW = T / 32;
+  __shared__ float s_w[NW];
+  __shared__ float s_c[C];
+  __shared__ __align__(8) uint64_t s_bar;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int q = (int)cluster.block_rank();
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const size_t row = blockIdx.x / C;
+  const int nvec = n / 4;
+  if (q == 0 && t == 0) {
+    mbar_init(&s_bar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(&s_bar, 4u * C);
+  }
+  // every CTA has started (and rank 0 initialised its barrier) once this
+  // arrive is matched; the wait comes before the push
+  cluster_arrive_relaxed();
+  const float4 *xr = reinterpret_cast<const float4 *>(x + row * n);
+  float p = 0.0f;
+  int vi = q * T + t;                              // this lane's vectors: vi, vi + 1024, ...
+  for (; vi + 7 * kLaneT < nvec; vi += 8 * kLaneT) {
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) v[k] = __ldcs(xr + vi + k * kLaneT);
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      p = __fadd_rn(p, v[k].x);
+      p = __fadd_rn(p, v[k].y);
+      p = __fadd_rn(p, v[k].z);
+      p = __fadd_rn(p, v[k].w);
+    }
+  }
+  for (; vi < nvec; vi += kLaneT) {
+    const float4 v = __ldcs(xr + vi);
+    p = __fadd_rn(p, v.x);
+    p = __fadd_rn(p, v.y);
+    p = __fadd_rn(p, v.z);
+    p = __fadd_rn(p, v.w);
+  }
+  const float g = warp_tree_sum(p);                // one 32-lane group
+  if (lane == 0) s_w[warp] = g;
+  __syncthreads();
+  float cv = 0.0f;                                 // the CTA's groups, perfect tree
+  if (warp == 0) {
+    cv = lane < NW ? s_w[lane] : 0.0f;
+#pragma unroll
+    for (int o = 1; o < NW; o <<= 1) cv = __fadd_rn(cv, __shfl_xor_sync(0xffffffffu, cv, o));
+  }
+  cluster_wait();
+  if (t == 0) st_async_f32(&s_c[q], &s_bar, 0u, cv);
+  if (q != 0 || warp != 0) return;
+  if (!mbar_wait_cluster(&s_bar, 0)) flag_error(status, BI_ERR_TIMEOUT);
+  float v = lane < C ? s_c[lane] : 0.0f;           // the top levels over the C CTAs
+#pragma unroll
+  for (int o = 1; o < C; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) out[row] = __fdiv_rn(v, (float)n);
 }
 
 // ======================================================================
@@ -375,7 +443,28 @@ extern "C" bi_status bi_mean(const float *x, float *out, int rows, int n, bi_str
   if (n % 4 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
   if (!bi_aligned16(x)) return BI_ERR_UNSUPPORTED_SHAPE;
   if (rows == 0) return BI_OK;
-  bi::mean_kernel<<<rows, bi::kMeanThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, out, n);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // few rows: a 16-CTA cluster per row (bit-neutral: the CTAs own subtrees)
+  if (rows <= bi::kMeanClusterRows) {
+    constexpr int C = 16;
+    auto kern = bi::mean_cluster_kernel<C>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)rows * C, 1, 1);
+    cfg.blockDim = dim3(bi::kLaneT / C, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    unsigned *status = bi::status_word();
+    return cudaLaunchKernelEx(&cfg, kern, x, out, n, status) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  }
+  bi::mean_kernel<<<rows, bi::kMeanThreads, 0, s>>>(x, out, n);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
