@@ -26,8 +26,8 @@
 // Kernel 1 (one CTA per chunk, kv head, sequence; 256 threads): every lane
 // loads one key row into registers and folds its scores; the PV sums read
 // V straight from global memory (a warp reads 128 contiguous bytes of one V
-// row per slot), so a CTA needs ~18 KB of shared memory and four share an
-// SM; the chunk partials (m_c, l_c, o_c) of the G query heads that share
+// row per slot), so a CTA needs little shared memory (18 KB at D = 128
+// with four query heads per kv head) and four share an SM there; the chunk partials (m_c, l_c, o_c) of the G query heads that share
 // the kv head go to the caller's workspace.  Kernel 2 (one CTA per query
 // head and sequence): the combine.
 #include "bimath.cuh"
