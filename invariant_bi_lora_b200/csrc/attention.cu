@@ -27,9 +27,10 @@
 // loads one key row into registers and folds its scores; the PV sums read
 // V straight from global memory (a warp reads 128 contiguous bytes of one V
 // row per slot), so a CTA needs little shared memory (18 KB at D = 128
-// with four query heads per kv head) and four share an SM there; the chunk partials (m_c, l_c, o_c) of the G query heads that share
-// the kv head go to the caller's workspace.  Kernel 2 (one CTA per query
-// head and sequence): the combine.
+// with four query heads per kv head) and four share an SM there; the chunk
+// partials (m_c, l_c, o_c) of the G query heads that share the kv head go
+// to the caller's workspace.  Kernel 2 (one CTA per query head and
+// sequence): the combine.
 #include "bimath.cuh"
 #include "tc.cuh"
 
