@@ -163,6 +163,20 @@ def test_mean_bit_exact_and_invariant(n, logits):
         assert np.array_equal(mean_gpu(x[:R]), full[:R])
 
 
+@pytest.mark.parametrize("n", [4, 100, 4096, 4100, 33000])
+def test_mean_few_rows_cluster_path(n):
+    """Up to 128 rows the mean runs one 16-CTA cluster per row (each CTA a
+    block of 64 lanes, a subtree): bitwise the oracle's canonical mean at
+    widths where some lanes hold no vector, one vector or many, and bitwise
+    the many-row kernel's rows."""
+    x = np.ascontiguousarray(synth.normal_f32((200, n), 1.0, seed=n + 1))
+    many = mean_gpu(x)                                  # 200 rows: one CTA per row
+    for R in (1, 3, 128):
+        few = mean_gpu(x[:R])
+        assert np.array_equal(few, oracle.mean_canon(x[:R]).view(np.uint32)), R
+        assert np.array_equal(few, many[:R]), R
+
+
 def test_mean_order_case():
     x = np.zeros((1, 8192), np.float32)
     x[0, 0], x[0, 4096], x[0, 4] = 1e8, 1.0, -1e8
