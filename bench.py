@@ -486,7 +486,10 @@ class Sweep:
       d4  segmented shrink (tree / atomic s=8, unsplit) and expand at
           r in {8, 16, 64}, M = 4096, 8 adapters;
       d5  tree GEMM K = 16384, N = 4096, M in {1, 128, 2048},
-          s in {1, 2, 4, 8} emulated shards (with the combine)."""
+          s in {1, 2, 4, 8} emulated shards (with the combine);
+      N2  the cross-rank combine by peer pointers (bi_tree_combine_peers)
+          over s separate partial buffers of M=2048 x N=4096 fp32, here all
+          on this GPU (standing in for s ranks' buffers), s in {2, 4, 8}."""
 
     def __init__(self, bi, synth, wl):
         self.bi, self.rows = bi, []
@@ -549,6 +552,13 @@ class Sweep:
                 self.add("d5", f"tree_gemm M={M} s={s}", {"M": M, "N": 4096, "K": 16384, "shards": s}, bound,
                          2 * M * 16384 + 2 * 4096 * 16384 + 4 * M * 4096, 2 * M * 4096 * 16384,
                          lambda A_=A_, C_=C_, s=s: bi.gemm_tree(A_, self.tw, C_, s, self.tws))
+        count = 2048 * 4096
+        self.peer_bufs = [torch.empty(count, dtype=torch.float32, device="cuda").normal_() for _ in range(8)]
+        self.peer_out = torch.empty(count, dtype=torch.float32, device="cuda")
+        for s_ in (2, 4, 8):
+            ptrs = [b.data_ptr() for b in self.peer_bufs[:s_]]
+            self.add("N2", f"tree_combine_peers s={s_}", {"count": count, "s": s_, "buffers": "local"}, "hbm",
+                     4 * count * (s_ + 1), 0, lambda ptrs=ptrs: bi.tree_combine_peers(ptrs, self.peer_out))
 
     def add(self, row, name, cfg, bound, nbytes, flops, fn):
         self.cases.append((row, name, cfg, bound, nbytes, flops, fn))
