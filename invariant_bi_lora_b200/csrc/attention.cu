@@ -84,6 +84,12 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
   const int c = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int L = max(0, min(p.lens[b], p.Lmax));      // a length past Lmax reads nothing beyond it
   const int j0 = c * kAttnChunk;
+  // one chunk per sequence at most (max_chunks == 1): this kernel writes the
+  // output itself, an empty sequence's included (see the end)
+  if (p.max_chunks == 1 && L == 0) {
+    for (int e = threadIdx.x; e < G * D; e += kAttnThreads) p.out[((size_t)b * p.Hq + hk * G) * D + e] = 0.0f;
+    return;
+  }
   if (j0 >= L) return;                              // past this sequence's chunks
   const int nj = min(kAttnChunk, L - j0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -242,6 +248,12 @@ attn_chunk_kernel(const __grid_constant__ AttnParams p) {
       for (int w = 1; w < QT; w <<= 1)
 #pragma unroll
         for (int e = 0; e + w < QT; e += 2 * w) r[e] = __fadd_rn(r[e], r[e + w]);
+      if (p.max_chunks == 1) {
+        // the combine over one chunk: weight bi_exp(0) = 1 exactly and no
+        // tree levels, so out = fl(o / l) -- the same bits as kernel 2
+        p.out[((size_t)b * p.Hq + hk * G + i) * D + d] = __fdiv_rn(r[0], l_i[i]);
+        continue;
+      }
       wsb[i * head_stride + 2 + d] = r[0];
       if (d == 0) {
         wsb[i * head_stride + 0] = m_i[i];
@@ -313,6 +325,7 @@ static bi_status attn_launch_d(const AttnParams &p, int G, cudaStream_t s) {
     default: return BI_ERR_UNSUPPORTED_SHAPE;
   }
   if (e != cudaSuccess) return BI_ERR_CUDA;
+  if (p.max_chunks == 1) return BI_OK;              // kernel 1 wrote the output
   attn_combine_kernel<D><<<dim3(p.Hq, p.B), D, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

@@ -49,6 +49,8 @@ def run(q, k, v, lens, scale):
     (4, 4, 4, 64, [256, 257, 0, 512]),
     (2, 8, 2, 256, [700, 33]),
     (2, 16, 2, 128, [4096, 1]),
+    (3, 8, 2, 128, [256, 0, 17]),          # one chunk at most: kernel 1 writes the output itself
+    (1, 4, 1, 64, [5]),
 ])
 def test_attention_bit_exact(B, Hq, Hkv, D, lens):
     Lmax = max(lens) if max(lens) > 0 else 1
